@@ -1,0 +1,6 @@
+"""fp64 CPU oracle for GPTQ layer quantization (test infrastructure only; see gptq_oracle)."""
+from .gptq_oracle import (  # noqa: F401
+    hessian_accumulate, hessian_finalize, hessian, damp, inverse_hessian_factor, quant_params,
+    quantize, gptq_quantize, gptq_quantize_unbatched, rtn_quantize, layer_error, gptq_layer,
+    check_shapes,
+)
