@@ -1,0 +1,413 @@
+"""Benchmark: GPTQ layer quantization of one 4096 x 4096 attention projection on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = the whole path for one layer on inputs already resident in HBM: S += X^T X over all
+262144 calibration tokens (S1), the damped inverse-Hessian factor (S2-S5) and the blocked column
+loop with lazy trailing updates (S6-S8), 4-bit, group 128, block 128. The metric is weights/s
+(rows * cols / step time), whole job over all ranks; `ms_per_step` is ms per layer.
+
+Multi-GPU: the layers are independent problems, so each rank quantizes its own layer (its own
+seeded inputs) with no collective on the data path ("scaling": "weak"); the timed region is
+bracketed by a barrier and device synchronizations and the max over ranks is reported.
+
+Extra keys: `roofline` for the dominant kernel (the tensor-core Hessian SYRK, timed live with CUDA
+events on its stream), `e2e` (the same work through the public API from pinned host buffers,
+copies included), `cpu_baseline` (the fp64 oracle on a bounded sample of the same workload,
+extrapolated; rank 0 at N=1 only), `clocks` (nvidia-smi sampled during the timed region) and
+`gpu_launches` (kernels the library enqueued inside the timed region).
+`--impl reference` times the fp64 CPU oracle on the same workload instead (bounded samples).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GPTQ layer quantize: weights/sec & ms per layer (4-bit g128); % of roofline"
+UNIT = "weights/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=10)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--tokens", type=int, default=0,
+                   help="override the calibration token count (profiling runs only; the line is "
+                        "then marked as not the configured workload)")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-sample-s", type=float, default=20.0)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload(tokens_override: int):
+    from post_weight_quantization_12_b200 import synth
+    spec = synth.ATTN
+    if tokens_override:
+        spec = synth.scaled_spec(spec, spec.rows, spec.cols, tokens_override)
+    return spec
+
+
+def config_dict(spec):
+    return {
+        "workload": f"attention projection: W {spec.rows}x{spec.cols} bf16 ~N(0,0.02^2); "
+                    f"X {spec.n_tokens} tokens x {spec.cols} bf16 Student-t(3), 1% channels x20; "
+                    f"{spec.bits}-bit asymmetric group {spec.group}, block {spec.block}, damp 1%",
+        "rows": spec.rows, "cols": spec.cols, "n_tokens": spec.n_tokens, "bits": spec.bits,
+        "group": spec.group, "block": spec.block,
+        "l2": f"inputs larger than L2: X is {spec.n_tokens * spec.cols * 2 / 1e9:.2f} GB, "
+              "read in full every step",
+    }
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks
+# ------------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        max_mhz = max(r[1] for r in rows)
+        pmax = max(r[2] for r in rows)
+        loaded = [r for r in rows if r[2] >= 0.5 * pmax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3])
+                          if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max_mhz,
+                "reasons": reasons, "samples": len(rows), "samples_under_load": len(loaded),
+                "power_w_max": pmax}
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle on a bounded sample
+# ------------------------------------------------------------------------------------------------
+
+def oracle_sample(W_np, X_np, spec, budget_s: float):
+    """Time the fp64 oracle stage by stage on a sample of the workload and extrapolate to the full
+    layer: S1 on a token subsample (time ~ tokens), S2-S5 in full, S6-S8 on a row subsample (rows
+    are independent given R; time ~ rows). Returns (seconds for the full layer, description)."""
+    import numpy as np
+    import oracle
+    cols = spec.cols
+    n_tok = X_np.shape[0]
+    t0 = time.perf_counter()
+    S = np.zeros((cols, cols))
+    oracle.hessian_accumulate(S, X_np)
+    t_s1 = time.perf_counter() - t0
+    H = oracle.hessian_finalize(S, n_tok)
+    t0 = time.perf_counter()
+    fac = oracle.inverse_hessian_factor(H, spec.damp)
+    t_s25 = time.perf_counter() - t0
+    r_sub = W_np.shape[0]
+    t0 = time.perf_counter()
+    oracle.gptq_quantize(W_np, fac["R"], spec.bits, spec.group, spec.block)
+    t_s68 = time.perf_counter() - t0
+    full = t_s1 * (spec.n_tokens / n_tok) + t_s25 + t_s68 * (spec.rows / r_sub)
+    desc = (f"S1 on {n_tok} of {spec.n_tokens} tokens ({t_s1:.2f} s, x{spec.n_tokens / n_tok:g}); "
+            f"S2-S5 in full at {cols}x{cols} ({t_s25:.2f} s); S6-S8 on {r_sub} of {spec.rows} rows "
+            f"({t_s68:.2f} s, x{spec.rows / r_sub:g}); extrapolated {full:.1f} s per layer")
+    return full, desc, t_s1 + t_s25 + t_s68
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def sample_sizes(spec, budget_s: float):
+    # chosen so the three stages take roughly budget_s together on a many-core host
+    n_tok = 8192 if budget_s >= 10 else 2048
+    r_sub = 64 if budget_s >= 10 else 16
+    return n_tok, r_sub
+
+
+# ------------------------------------------------------------------------------------------------
+# reference arm: the oracle itself
+# ------------------------------------------------------------------------------------------------
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    from post_weight_quantization_12_b200 import synth
+    spec = workload(args.tokens)
+    n_tok, r_sub = sample_sizes(spec, args.cpu_sample_s)
+    sub = synth.scaled_spec(spec, r_sub, spec.cols, n_tok)
+    W = synth.weights_np(sub, args.seed)
+    X = synth.inputs_np(sub, args.seed)
+    times = []
+    for i in range(args.warmup + args.steps):
+        full, desc, spent = oracle_sample(W, X, spec, args.cpu_sample_s)
+        if i >= args.warmup:
+            times.append(full)
+    t = statistics.mean(times)
+    value = spec.rows * spec.cols / t
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded; numpy draws of the same recipe)", "config": config_dict(spec),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+# our arm
+# ------------------------------------------------------------------------------------------------
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from post_weight_quantization_12_b200 import _lib, api, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    peaks, peaks_src = load_peaks()
+    spec = workload(args.tokens)
+    seed = args.seed + 1000 * rank
+    rows, cols, n = spec.rows, spec.cols, spec.n_tokens
+
+    X = synth.inputs_torch(spec, seed, dev)
+    W = synth.weights_torch(spec, seed, dev)
+    S = torch.empty(cols, cols, device=dev)
+    R = torch.empty(cols, cols, device=dev)
+    G = 1 if spec.group <= 0 else cols // spec.group
+    W_hat = torch.empty(rows, cols, device=dev)
+    codes = torch.empty(rows, cols, device=dev, dtype=torch.uint8)
+    scales = torch.empty(rows, G, device=dev)
+    zeros = torch.empty(rows, G, device=dev, dtype=torch.uint8)
+    err_sq = torch.empty(rows, device=dev)
+    ws_p = torch.empty(_lib.workspace_size(_lib.GPTQ_WS_PREPARE, 0, cols, 0), device=dev,
+                       dtype=torch.uint8)
+    ws_q = torch.empty(_lib.workspace_size(_lib.GPTQ_WS_QUANTIZE, rows, cols, spec.block),
+                       device=dev, dtype=torch.uint8)
+    info = torch.zeros(1, device=dev, dtype=torch.int32)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        S.zero_()
+        if ev is not None:
+            ev[0].record(stream)
+        _lib.hessian_accumulate(S, X, info, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        _lib.prepare_hinv(S, R, n, spec.damp, ws_p, info, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        _lib.quantize_layer(W, R, spec.bits, spec.group, spec.block, W_hat, codes, scales, zeros,
+                            err_sq, ws_q, info, stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(info.item()) != 0:
+        raise RuntimeError(f"device status {int(info.item())} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    clocks = ClockSampler(local) if rank == 0 else None
+    if clocks:
+        clocks.start()
+        time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    launches0 = _lib.kernel_launches()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    launches = _lib.kernel_launches() - launches0
+    if world > 1:
+        dist.barrier()
+    clock_rec = clocks.stop() if clocks else None
+    elapsed_ms = t_start.elapsed_time(t_end)
+    s1 = [e[0].elapsed_time(e[1]) for e in evs]
+    s25 = [e[1].elapsed_time(e[2]) for e in evs]
+    s68 = [e[2].elapsed_time(e[3]) for e in evs]
+    if int(info.item()) != 0:
+        raise RuntimeError(f"device status {int(info.item())} in the timed region")
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+        c = torch.tensor([launches], device=dev, dtype=torch.int64)
+        dist.all_reduce(c, op=dist.ReduceOp.SUM)
+        launches = int(c.item())
+
+    ms_per_step = elapsed_ms / args.steps
+    value = world * rows * cols * args.steps / (elapsed_ms / 1e3)
+
+    # roofline of the dominant kernel: the SYRK (S1 is exactly one kernel launch)
+    t_syrk = statistics.mean(s1) / 1e3
+    flops = cols * (cols + 1) * n            # symmetric half of X^T X, 2 flops per multiply-add
+    achieved = flops / t_syrk / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": "hessian_syrk_bf16_tc",
+                "peak_source": f"{peaks_src} bf16 sustained (kernel timed inside a long step)",
+                "work": f"{flops:.4g} flop per launch = cols*(cols+1)*n_tokens"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16/f32",
+        "data": "synthetic (seeded device draws; no model weights or calibration text)",
+        "config": config_dict(spec),
+        "stages_ms": {"S1_hessian": statistics.mean(s1), "S2_S5_factor": statistics.mean(s25),
+                      "S6_S8_quantize": statistics.mean(s68)},
+        "roofline": roofline, "gpu_launches": launches, "clocks": clock_rec,
+    }
+    if args.tokens:
+        line["note"] = "token count overridden for profiling: not the configured workload"
+
+    # end to end through the public API from pinned host buffers
+    if not args.no_e2e:
+        Xh = X.cpu().pin_memory()
+        Wh = W.cpu().pin_memory()
+        q = api.LayerQuantizer(cols, device=dev, damp_rel=spec.damp)
+
+        def e2e_step():
+            q.reset()
+            q.add_batch(Xh)
+            q.prepare()
+            return q.quantize(Wh, spec.bits, spec.group, spec.block, to_host=True)
+
+        for _ in range(min(2, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize(dev)
+        k_e2e = max(1, min(3, args.steps))
+        if world > 1:
+            dist.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(k_e2e):
+            out = e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        e_ms = a.elapsed_time(b)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
+        d2h = sum(t.numel() * t.element_size() for t in (out.codes, out.scales, out.zeros,
+                                                         out.W_hat, out.err_sq))
+        line["e2e"] = {"value": world * rows * cols * k_e2e / (e_ms / 1e3), "unit": UNIT,
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "steps": k_e2e, "ms_per_step": e_ms / k_e2e}
+        del Xh, Wh
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        n_tok, r_sub = sample_sizes(spec, args.cpu_sample_s)
+        Xs = X[:n_tok].float().cpu().numpy()
+        Ws = W[:r_sub].float().cpu().numpy()
+        full, desc, spent = oracle_sample(Ws, Xs, spec, args.cpu_sample_s)
+        line["cpu_baseline"] = {"value": rows * cols / full, "unit": UNIT,
+                                "cores": cpu_threads(), "kind": "oracle", "sample": desc,
+                                "sample_wall_s": spent}
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

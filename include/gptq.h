@@ -1,0 +1,181 @@
+/*
+ * gptq.h -- C ABI of libgptq_b200: GPTQ layer quantization on NVIDIA B200 (sm_100a).
+ *
+ * The problem: for a linear layer with weights W (rows x cols) and calibration inputs X, find a
+ * k-bit W_hat that keeps ||W X - W_hat X||^2 small ("GPTQ second-order quantization" blog, section
+ * "The objective is layer output, not weight distance"), by rounding columns in a fixed order and
+ * moving the not-yet-rounded columns to absorb each rounding error, with the inverse-Hessian
+ * information read from a Cholesky factor ("Part 3: Adaptive Rounding: GPTQ", "Algorithm GPTQ").
+ *
+ * Three calls make the path, in this order:
+ *   1. gptq_hessian_accumulate  S += X^T X over chunks of calibration tokens        (step S1)
+ *   2. gptq_prepare_hinv        H = 2S/N; damping; upper factor R of (H+lambda I)^-1 (S2-S5)
+ *   3. gptq_quantize_layer      blocked column loop with lazy trailing updates       (S6-S8)
+ *
+ * Conventions for every call:
+ *   - Pointers named *_dev, and every matrix argument, are DEVICE pointers to caller-owned
+ *     memory (e.g. torch CUDA tensors). The library never allocates, frees or keeps them.
+ *   - Matrices are row-major. "ld" arguments are leading dimensions in elements.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream). Every call only enqueues work
+ *     on that stream and returns; it never synchronizes.
+ *   - The return value reports argument and launch errors found on the host, before or while
+ *     enqueueing; on any error other than GPTQ_OK nothing further was enqueued.
+ *   - Conditions found on the device are written to the caller's int32 status word `info_dev`
+ *     (see GPTQ_INFO_*). The caller sets it to 0 once; kernels only ever replace 0 by the first
+ *     error they detect, and the library never clears it. Read it after synchronizing.
+ *   - Calls on distinct buffers may run concurrently on different streams.
+ */
+#ifndef GPTQ_B200_H
+#define GPTQ_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum gptq_status {
+  GPTQ_OK = 0,
+  GPTQ_EINVAL = 1,         /* an argument is out of range, misaligned or inconsistent */
+  GPTQ_ENOTPD = 2,         /* (from gptq_info_status) a factorization met a non-positive pivot */
+  GPTQ_ECUDA = 3,          /* a CUDA runtime call failed (launch, attribute, driver entry point) */
+  GPTQ_EUNSUPPORTED = 4,   /* a valid request this build does not implement (e.g. dtype/size) */
+  GPTQ_ETIMEOUT = 5,       /* (from gptq_info_status) a bounded device-side wait expired */
+  GPTQ_EWORKSPACE = 6      /* workspace missing or smaller than gptq_workspace_size() */
+} gptq_status;
+
+typedef enum gptq_dtype { GPTQ_BF16 = 0, GPTQ_FP32 = 1 } gptq_dtype;
+
+/* Values the kernels write into *info_dev (the first one detected wins). */
+#define GPTQ_INFO_OK 0
+/* 1 .. cols:        H + lambda I is not positive definite; value = 1-based pivot index (S3). */
+/* cols+1 .. 2*cols: the formed inverse is not positive definite; value - cols = pivot (S5). */
+#define GPTQ_INFO_TIMEOUT (-1)        /* a bounded wait inside a kernel expired */
+#define GPTQ_INFO_BAD_HESSIAN (-2)    /* mean(diag H) <= 0 or not finite: nothing to damp */
+
+/* Which workspace gptq_workspace_size() reports. */
+#define GPTQ_WS_PREPARE 1
+#define GPTQ_WS_QUANTIZE 2
+
+/*
+ * S1 -- proxy Hessian accumulation: S += X^T X.
+ *
+ * Source: "Part 2: Adaptive Rounding: Optimal Brain Quantizer (OBQ)", section "Goal" (the input
+ * covariance E[x x^T] is the proxy Hessian); "Part 3: Adaptive Rounding: GPTQ", "Algorithm GPTQ"
+ * (H = X X^T + lambda I, X stored there as cols x tokens).
+ *
+ *   S_dev      float32 [cols x cols], ld = cols. Only the lower triangle (i >= j) is accumulated
+ *              and meaningful; the strict upper triangle is scratch (it may receive partial sums).
+ *              The caller zeroes S once before the first chunk.
+ *   X_dev      calibration inputs, TOKEN-major: [n_tokens x ldx], columns 0..cols-1 used.
+ *              GPTQ_BF16: tensor-core path (tcgen05, bf16 products, fp32 accumulation);
+ *                requires cols % 8 == 0, ldx % 8 == 0 and a 16-byte aligned X_dev.
+ *              GPTQ_FP32: fp32 CUDA-core path (exact fp32 products and sums), any cols.
+ *   n_tokens   tokens in this chunk (0 = nothing to do). Call repeatedly to stream chunks; the
+ *              total over all calls is the N given to gptq_prepare_hinv.
+ *   info_dev   status word (GPTQ_INFO_TIMEOUT if a pipeline wait expires).
+ * Errors: GPTQ_EINVAL for null pointers, cols <= 0, ldx < cols, n_tokens < 0 or alignment.
+ */
+gptq_status gptq_hessian_accumulate(float* S_dev, int64_t cols, const void* X_dev,
+                                    gptq_dtype x_dtype, int64_t n_tokens, int64_t ldx,
+                                    int32_t* info_dev, void* stream);
+
+/*
+ * S2-S5 -- damped inverse-Hessian factor.
+ *
+ * Source: "GPTQ second-order quantization" blog, sections "The objective is layer output"
+ * (H = 2 X X^T) and "3. Cholesky reformulation" (damping of about 1 % of the mean Hessian
+ * diagonal; Cholesky factor computed once); "Part 3: Adaptive Rounding: GPTQ", "Observation 3:
+ * The Cholesky Reformulation" and "Algorithm GPTQ" (Cholesky of H^-1, one factor row read per
+ * column). The route: H_d = H + lambda I = L L^T (blocked Cholesky), L^-1 (triangular inverse),
+ * H_d^-1 = L^-T L^-1, H_d^-1 = R^T R with R upper (Cholesky of the inverse).
+ *
+ *   S_H_dev    in:  S from gptq_hessian_accumulate (lower triangle read).
+ *              out: H = (2 / n_total) S, both triangles, undamped (kept for the layer metric).
+ *   R_dev      out: float32 [cols x cols], ld = cols: R upper triangular with positive diagonal,
+ *              (H + lambda I)^-1 = R^T R, strictly lower part set to 0.
+ *   n_total    total number of calibration tokens accumulated into S (> 0).
+ *   damp_rel   lambda = damp_rel * mean(diag H) (the pages use 0.01); must be >= 0.
+ *   ws_dev     device workspace of at least gptq_workspace_size(GPTQ_WS_PREPARE, 0, cols, 0)
+ *              bytes, 256-byte aligned; contents on entry do not matter.
+ *   info_dev   status word: pivot codes (see GPTQ_INFO_*), GPTQ_INFO_BAD_HESSIAN.
+ * Errors: GPTQ_EINVAL (null pointers, cols <= 0, n_total <= 0, damp_rel < 0), GPTQ_EWORKSPACE.
+ */
+gptq_status gptq_prepare_hinv(float* S_H_dev, float* R_dev, int64_t cols, int64_t n_total,
+                              float damp_rel, void* ws_dev, size_t ws_bytes, int32_t* info_dev,
+                              void* stream);
+
+/*
+ * S6-S8 -- the GPTQ column loop with lazy batch updates.
+ *
+ * Source: "Part 3: Adaptive Rounding: GPTQ", "Observation 1" (one fixed left-to-right column
+ * order shared by all rows), "Observation 2: Lazy Batch Updates" (B columns processed on chip,
+ * later columns updated by one matrix product per block) and "Algorithm GPTQ"; the update
+ * W[:, B:] -= E R[B, B:] as the Vietnamese edition of the GPTQ blog writes it ("2. Lazy batch
+ * update"); the design table (asymmetric uniform, 3-4 bit, per row or group 128) and the blog's
+ * "Group-wise quantization". For each block of B columns [b0, b1) and each column j in order:
+ *     q_j   = clamp(rint(w_j / s) + z, 0, 2^bits - 1)           (float32, round half to even)
+ *     what_j = s * (q_j - z)
+ *     e_j   = (w_j - what_j) / R[j][j];   E[:, j - b0] = e_j
+ *     W[:, j+1 : b1] -= e_j * R[j, j+1 : b1]                    (in-block, on chip)
+ *   then W[:, b1:] -= E * R[b0:b1, b1:]                           (lazy trailing update)
+ * Grid of a row or group: lo = min(0, min v), hi = max(0, max v) (an all-zero v uses [-1, 1]),
+ * s = (hi - lo) / (2^bits - 1), z = clamp(rint(-lo / s), 0, 2^bits - 1), each step rounded once
+ * in float32. Per-row grids come from the ORIGINAL weights; group grids from the current
+ * (already compensated) weights when the group's first column is reached.
+ *
+ *   W_dev      original weights [rows x ldw] (GPTQ_BF16 or GPTQ_FP32); not modified.
+ *   R_dev      float32 [cols x cols] from gptq_prepare_hinv (upper triangle read).
+ *   bits       2..8.
+ *   group      -1 (one grid per row) or a group size g >= 1 with cols % g == 0 and either
+ *              g % block == 0 or block % g == 0.
+ *   block      B, one of 32, 64, 128.
+ *   W_hat_dev  out: float32 [rows x cols], ld = cols: the dequantized weights s * (q - z).
+ *              Also the working buffer of the loop.
+ *   codes_dev  out: uint8 [rows x cols], ld = cols, values 0 .. 2^bits - 1 (unpacked).
+ *   scales_dev out: float32 [rows x G]; zeros_dev out: uint8 [rows x G]; G = 1 (per-row) or
+ *              cols / group.
+ *   err_sq_dev out (may be NULL): float32 [rows], sum over j of e_j^2 (the damped proxy loss of
+ *              the row, since W_hat - W = -e R and (H + lambda I) = R^-1 R^-T).
+ *   ws_dev     device workspace of gptq_workspace_size(GPTQ_WS_QUANTIZE, rows, cols, block)
+ *              bytes, 256-byte aligned.
+ *   info_dev   status word.
+ * Errors: GPTQ_EINVAL (shapes, bits, group/block rules, null pointers), GPTQ_EWORKSPACE.
+ */
+gptq_status gptq_quantize_layer(const void* W_dev, gptq_dtype w_dtype, int64_t rows, int64_t cols,
+                                int64_t ldw, const float* R_dev, int bits, int group, int block,
+                                float* W_hat_dev, uint8_t* codes_dev, float* scales_dev,
+                                uint8_t* zeros_dev, float* err_sq_dev, void* ws_dev,
+                                size_t ws_bytes, int32_t* info_dev, void* stream);
+
+/* Workspace bytes needed by one call (GPTQ_WS_PREPARE or GPTQ_WS_QUANTIZE); 0 for bad input. */
+size_t gptq_workspace_size(int which, int64_t rows, int64_t cols, int block);
+
+/* Maps a status word read back from the device to a gptq_status (0 -> GPTQ_OK,
+   pivot codes -> GPTQ_ENOTPD, GPTQ_INFO_TIMEOUT -> GPTQ_ETIMEOUT, others -> GPTQ_EINVAL). */
+gptq_status gptq_info_status(int32_t info);
+
+/* Static, human-readable name of a status code. */
+const char* gptq_status_string(int status);
+
+/* Number of CUDA kernels this library has enqueued since it was loaded, over all calls and
+   devices (a diagnostic counter; copies and memsets are not counted). */
+uint64_t gptq_kernel_launches(void);
+
+/*
+ * Self-test of the bounded device waits (no counterpart on the pages). Enqueues one CTA that
+ * waits on a shared-memory barrier nothing will ever arrive on, giving up after limit_ms
+ * milliseconds (1..10000); on giving up it writes GPTQ_INFO_TIMEOUT into *info_dev and returns,
+ * leaving the context usable. Lets callers check that a lost wait ends as a status, not a hang.
+ */
+gptq_status gptq_selftest_wait_timeout(int32_t* info_dev, int limit_ms, void* stream);
+
+/* Library version, "major.minor.patch". */
+const char* gptq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GPTQ_B200_H */

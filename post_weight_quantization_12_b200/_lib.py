@@ -1,0 +1,141 @@
+"""ctypes binding of libgptq_b200.so: argument marshalling only.
+
+Every function here passes raw device pointers, sizes and the current CUDA stream to the C ABI
+declared in include/gptq.h; all arithmetic runs in the library's CUDA kernels. Loading fails
+loudly when the shared library has not been built -- there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libgptq_b200.so")
+
+GPTQ_OK, GPTQ_EINVAL, GPTQ_ENOTPD, GPTQ_ECUDA, GPTQ_EUNSUPPORTED, GPTQ_ETIMEOUT, \
+    GPTQ_EWORKSPACE = range(7)
+GPTQ_BF16, GPTQ_FP32 = 0, 1
+GPTQ_INFO_TIMEOUT = -1
+GPTQ_INFO_BAD_HESSIAN = -2
+GPTQ_WS_PREPARE, GPTQ_WS_QUANTIZE = 1, 2
+
+# name -> (restype, argtypes)
+_P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "gptq_hessian_accumulate": (_I32, [_P, _I64, _P, _I32, _I64, _I64, _P, _P]),
+    "gptq_prepare_hinv": (_I32, [_P, _P, _I64, _I64, _F, _P, _SZ, _P, _P]),
+    "gptq_quantize_layer": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _I32, _I32, _P, _P, _P,
+                                   _P, _P, _P, _SZ, _P, _P]),
+    "gptq_workspace_size": (_SZ, [_I32, _I64, _I64, _I32]),
+    "gptq_info_status": (_I32, [ctypes.c_int32]),
+    "gptq_status_string": (ctypes.c_char_p, [_I32]),
+    "gptq_version": (ctypes.c_char_p, []),
+    "gptq_kernel_launches": (ctypes.c_uint64, []),
+    "gptq_selftest_wait_timeout": (_I32, [_P, _I32, _P]),
+}
+
+_lib = None
+
+
+class GPTQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)}")
+
+
+def load():
+    """Load libgptq_b200.so (built in-tree); raises if it is missing."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m post_weight_quantization_12_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return load().gptq_status_string(int(status)).decode()
+
+
+def info_status(info: int) -> int:
+    return int(load().gptq_info_status(int(info)))
+
+
+def workspace_size(which: int, rows: int, cols: int, block: int) -> int:
+    return int(load().gptq_workspace_size(which, rows, cols, block))
+
+
+def kernel_launches() -> int:
+    """Kernels the library has enqueued since it was loaded (diagnostic counter)."""
+    return int(load().gptq_kernel_launches())
+
+
+def selftest_wait_timeout(info, limit_ms: int, stream=None):
+    """Enqueue a bounded wait that nothing will satisfy; it must end with GPTQ_INFO_TIMEOUT."""
+    _check(load().gptq_selftest_wait_timeout(_ptr(info), int(limit_ms), _stream(stream)),
+           "gptq_selftest_wait_timeout")
+
+
+def _check(st: int, where: str):
+    if st != GPTQ_OK:
+        raise GPTQError(st, where)
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _dtype_code(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return GPTQ_BF16
+    if t.dtype == torch.float32:
+        return GPTQ_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _row_major_ld(t, name):
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D tensor with unit column stride")
+    return t.stride(0)
+
+
+def hessian_accumulate(S, X, info, stream=None):
+    """S[cols, cols] (fp32) += X^T X for token-major X[n_tokens, >= cols] (bf16 or fp32)."""
+    ldx = _row_major_ld(X, "X")
+    st = load().gptq_hessian_accumulate(_ptr(S), S.shape[0], _ptr(X), _dtype_code(X), X.shape[0],
+                                        ldx, _ptr(info), _stream(stream))
+    _check(st, "gptq_hessian_accumulate")
+
+
+def prepare_hinv(S_H, R, n_total, damp_rel, ws, info, stream=None):
+    """S_H: S in, H = 2S/N out (both triangles); R: upper factor of (H + lambda I)^-1."""
+    st = load().gptq_prepare_hinv(_ptr(S_H), _ptr(R), S_H.shape[0], int(n_total), float(damp_rel),
+                                  _ptr(ws), ws.numel() * ws.element_size(), _ptr(info),
+                                  _stream(stream))
+    _check(st, "gptq_prepare_hinv")
+
+
+def quantize_layer(W, R, bits, group, block, W_hat, codes, scales, zeros, err_sq, ws, info,
+                   stream=None):
+    """GPTQ column loop over W[rows, cols] with the factor R; outputs are caller tensors."""
+    ldw = _row_major_ld(W, "W")
+    st = load().gptq_quantize_layer(
+        _ptr(W), _dtype_code(W), W.shape[0], W.shape[1], ldw, _ptr(R), int(bits), int(group),
+        int(block), _ptr(W_hat), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(err_sq), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(info), _stream(stream))
+    _check(st, "gptq_quantize_layer")

@@ -1,0 +1,100 @@
+"""User-facing layer quantizer: allocates device buffers with PyTorch and calls the C ABI.
+
+    q = LayerQuantizer(cols, device="cuda")
+    for chunk in calibration_chunks:          # token-major [n, cols] bf16/fp32, host or device
+        q.add_batch(chunk)
+    out = q.quantize(W, bits=4, group=128, block=128)   # W [rows, cols] host or device
+
+Host tensors are copied to the device (pinned-memory, non-blocking) before the call; outputs stay
+on the device unless `to_host=True`. PyTorch only provides memory and streams here; every step of
+the method runs in the library's kernels.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+from . import _lib
+
+
+@dataclass
+class QuantizedLayer:
+    codes: torch.Tensor      # uint8 [rows, cols]
+    scales: torch.Tensor     # fp32 [rows, G]
+    zeros: torch.Tensor      # uint8 [rows, G]
+    W_hat: torch.Tensor      # fp32 [rows, cols] dequantized weights
+    err_sq: torch.Tensor     # fp32 [rows] sum of squared scaled errors
+    info: int                # device status word after the call
+
+
+class LayerQuantizer:
+    """Streams calibration chunks into S, then factors and quantizes one layer (or several layers
+    that share the same inputs, e.g. q/k/v projections)."""
+
+    def __init__(self, cols: int, device="cuda", damp_rel: float = 0.01, stream=None):
+        self.cols = int(cols)
+        self.device = torch.device(device)
+        self.damp_rel = float(damp_rel)
+        self.stream = stream
+        self.S = torch.zeros(self.cols, self.cols, device=self.device, dtype=torch.float32)
+        self.info = torch.zeros(1, device=self.device, dtype=torch.int32)
+        self.n_total = 0
+        self.R = None
+
+    def reset(self):
+        """Start a new layer: S = 0, no tokens, no factor."""
+        self.S.zero_()
+        self.info.zero_()
+        self.n_total = 0
+        self.R = None
+
+    def _on_device(self, t: torch.Tensor) -> torch.Tensor:
+        if t.device == self.device:
+            return t
+        if t.device.type == "cpu":
+            if not t.is_pinned():
+                t = t.pin_memory()
+            return t.to(self.device, non_blocking=True)
+        return t.to(self.device)
+
+    def add_batch(self, X: torch.Tensor):
+        """S += X^T X for token-major calibration inputs X [n_tokens, cols] (bf16 or fp32)."""
+        X = self._on_device(X)
+        _lib.hessian_accumulate(self.S, X, self.info, self.stream)
+        self.n_total += X.shape[0]
+
+    def prepare(self):
+        """H = 2S/N (kept in self.S) and R, the upper factor of (H + lambda I)^-1."""
+        ws = torch.empty(_lib.workspace_size(_lib.GPTQ_WS_PREPARE, 0, self.cols, 0),
+                         device=self.device, dtype=torch.uint8)
+        self.R = torch.empty(self.cols, self.cols, device=self.device, dtype=torch.float32)
+        _lib.prepare_hinv(self.S, self.R, self.n_total, self.damp_rel, ws, self.info, self.stream)
+        return self.R
+
+    @property
+    def H(self):
+        return self.S
+
+    def quantize(self, W: torch.Tensor, bits: int = 4, group: int = 128, block: int = 128,
+                 to_host: bool = False) -> QuantizedLayer:
+        if self.R is None:
+            self.prepare()
+        W = self._on_device(W)
+        rows, cols = W.shape
+        G = 1 if group <= 0 else cols // group
+        dev = self.device
+        W_hat = torch.empty(rows, cols, device=dev, dtype=torch.float32)
+        codes = torch.empty(rows, cols, device=dev, dtype=torch.uint8)
+        scales = torch.empty(rows, G, device=dev, dtype=torch.float32)
+        zeros = torch.empty(rows, G, device=dev, dtype=torch.uint8)
+        err_sq = torch.empty(rows, device=dev, dtype=torch.float32)
+        ws = torch.empty(_lib.workspace_size(_lib.GPTQ_WS_QUANTIZE, rows, cols, block),
+                         device=dev, dtype=torch.uint8)
+        _lib.quantize_layer(W, self.R, bits, group, block, W_hat, codes, scales, zeros, err_sq, ws,
+                            self.info, self.stream)
+        info = int(self.info.item())
+        if to_host:
+            codes, scales, zeros, W_hat, err_sq = (t.cpu() for t in (codes, scales, zeros, W_hat,
+                                                                     err_sq))
+        return QuantizedLayer(codes, scales, zeros, W_hat, err_sq, info)

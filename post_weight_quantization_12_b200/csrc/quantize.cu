@@ -1,0 +1,278 @@
+// S6-S8 -- the GPTQ column loop with lazy batch updates.
+//
+// "Part 3: Adaptive Rounding: GPTQ": "Observation 1" (one left-to-right column order shared by
+// all rows, so rows run in parallel against one factor), "Observation 2: Lazy Batch Updates"
+// (a block of B columns is processed on chip and the later columns get one matrix product per
+// block), "Algorithm GPTQ"; the Vietnamese edition of the GPTQ blog, "2. Lazy batch update"
+// (W[:, B:] -= E R[B, B:]); the design table and the blog's "Group-wise quantization"
+// (asymmetric uniform grid per row or per group).
+//
+// Column loop layout: 8 consecutive lanes own one weight row; lane t of the row holds columns
+// [t * B/8, (t + 1) * B/8) of the current block in registers. The block's B x B corner of R sits
+// in shared memory with its diagonal and lower part replaced by zeros, so the in-block update
+// w[c] -= e * R[j][c] needs no mask (columns at or before j are left untouched). Every lane of a
+// row computes the same code for column j from the value broadcast by its owner lane, so no
+// further communication is needed per column.
+#include <cuda_bf16.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gptq {
+
+constexpr int kTPR = 8;  // lanes per weight row
+
+// Grid of the asymmetric min/max quantizer (IEEE float32, each step rounded once).
+__device__ __forceinline__ void grid_params(float lo, float hi, float maxq, float& s, float& z) {
+  lo = fminf(lo, 0.f);
+  hi = fmaxf(hi, 0.f);
+  if (lo == hi) { lo = -1.f; hi = 1.f; }
+  s = __fdiv_rn(__fsub_rn(hi, lo), maxq);
+  z = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), maxq);
+}
+
+template <typename T>
+__device__ __forceinline__ float load_w(const T* p);
+template <>
+__device__ __forceinline__ float load_w<float>(const float* p) { return *p; }
+template <>
+__device__ __forceinline__ float load_w<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
+template <typename T>
+__global__ void convert_kernel(const T* __restrict__ W, int64_t ldw, float* __restrict__ Wh,
+                               int64_t rows, int64_t cols) {
+  const int64_t total = rows * cols;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = e / cols, c = e - r * cols;
+    Wh[e] = load_w<T>(W + r * ldw + c);
+  }
+}
+
+// One warp per row: grid of columns [c0, c0 + len) of the current weights.
+__global__ void params_kernel(const float* __restrict__ Wh, int64_t rows, int64_t cols, int64_t c0,
+                              int64_t len, int bits, float* scales, uint8_t* zeros, int G, int gi) {
+  const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  float lo = 0.f, hi = 0.f;
+  const float* w = Wh + row * cols + c0;
+  for (int64_t c = lane; c < len; c += 32) {
+    const float v = w[c];
+    lo = fminf(lo, v);
+    hi = fmaxf(hi, v);
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0) {
+    float s, z;
+    grid_params(lo, hi, static_cast<float>((1 << bits) - 1), s, z);
+    scales[row * G + gi] = s;
+    zeros[row * G + gi] = static_cast<uint8_t>(z);
+  }
+}
+
+// One block of B columns [b0, b0 + nb) for every row.
+//   group_mode: 0 = grid given per row (scales[row*G + gi_fixed]);
+//               1 = groups of `group` columns inside the block, grids computed here.
+template <int B>
+__global__ void __launch_bounds__(128)
+column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const float* __restrict__ R,
+                   int b0, int nb, int bits, int group, int group_mode, int gi_fixed,
+                   float* __restrict__ scales, uint8_t* __restrict__ zeros, int G,
+                   uint8_t* __restrict__ codes, float* __restrict__ E, float* __restrict__ err_sq) {
+  constexpr int CPL = B / kTPR;  // columns per lane
+  extern __shared__ __align__(16) float qsm[];
+  float (*Rz)[B] = reinterpret_cast<float (*)[B]>(qsm);
+  float* inv_d = qsm + B * B;
+  for (int e = threadIdx.x; e < B * B; e += blockDim.x) {
+    const int i = e / B, j = e % B;
+    Rz[i][j] = (i < nb && j < nb && j > i) ? R[(b0 + i) * cols + b0 + j] : 0.f;
+  }
+  for (int i = threadIdx.x; i < B; i += blockDim.x)
+    inv_d[i] = (i < nb) ? 1.f / R[(b0 + i) * cols + b0 + i] : 0.f;
+  __syncthreads();
+
+  const int lane = threadIdx.x & 31;
+  const int sub = lane & (kTPR - 1);          // position within the row's lane group
+  const int base_lane = lane & ~(kTPR - 1);
+  const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x / kTPR) + threadIdx.x / kTPR;
+  const bool valid = row < rows;
+  const int c_first = sub * CPL;              // first block column this lane holds
+
+  float v[CPL];
+  uint8_t q8[CPL];
+  float err[CPL];
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) {
+    const int c = c_first + k;
+    v[k] = (valid && c < nb) ? Wh[row * cols + b0 + c] : 0.f;
+    q8[k] = 0;
+    err[k] = 0.f;
+  }
+  const float maxq = static_cast<float>((1 << bits) - 1);
+  float s = 1.f, z = 0.f;
+  if (group_mode == 0 && valid) {
+    s = scales[row * G + gi_fixed];
+    z = static_cast<float>(zeros[row * G + gi_fixed]);
+  }
+
+  for (int o = 0; o < kTPR; ++o) {
+#pragma unroll
+    for (int kk = 0; kk < CPL; ++kk) {
+      const int j = o * CPL + kk;
+      if (j < nb) {
+        if (group_mode == 1 && (j % group) == 0) {
+          float lo = 0.f, hi = 0.f;
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            const int c = c_first + k;
+            if (c >= j && c < j + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
+          }
+#pragma unroll
+          for (int off = kTPR / 2; off > 0; off >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+          }
+          grid_params(lo, hi, maxq, s, z);
+          if (valid && sub == 0) {
+            const int gi = (b0 + j) / group;
+            scales[row * G + gi] = s;
+            zeros[row * G + gi] = static_cast<uint8_t>(z);
+          }
+        }
+        const float w = __shfl_sync(0xffffffffu, v[kk], base_lane + o);
+        const float q = fminf(fmaxf(rintf(__fdiv_rn(w, s)) + z, 0.f), maxq);
+        const float wh = __fmul_rn(s, q - z);
+        const float e = __fmul_rn(__fsub_rn(w, wh), inv_d[j]);
+        if (sub == o) {
+          v[kk] = wh;
+          q8[kk] = static_cast<uint8_t>(q);
+          err[kk] = e;
+        }
+        const float* rrow = &Rz[j][c_first];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) v[k] = fmaf(-e, rrow[k], v[k]);
+      }
+    }
+  }
+
+  float sq = 0.f;
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) sq = fmaf(err[k], err[k], sq);
+#pragma unroll
+  for (int off = kTPR / 2; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+  if (!valid) return;
+#pragma unroll
+  for (int k = 0; k < CPL; ++k) {
+    const int c = c_first + k;
+    if (c < nb) {
+      Wh[row * cols + b0 + c] = v[k];
+      codes[row * cols + b0 + c] = q8[k];
+      E[row * B + c] = err[k];
+    }
+  }
+  if (sub == 0 && err_sq != nullptr) err_sq[row] += sq;
+}
+
+size_t quantize_workspace_bytes(int64_t rows, int64_t cols, int block) {
+  (void)cols;
+  return align_up(static_cast<size_t>(rows) * block * 4, 256);
+}
+
+template <int B>
+static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, const float* R, int b0,
+                                      int nb, int bits, int group, int group_mode, int gi_fixed,
+                                      float* scales, uint8_t* zeros, int G, uint8_t* codes,
+                                      float* E, float* err_sq, cudaStream_t stream) {
+  const int rows_per_cta = 128 / kTPR;
+  const int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
+  constexpr int smem = (B * B + B) * 4;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(column_loop_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+      return GPTQ_ECUDA;
+    attr_done = true;
+  }
+  column_loop_kernel<B><<<static_cast<unsigned>(grid), 128, smem, stream>>>(
+      Wh, rows, cols, R, b0, nb, bits, group, group_mode, gi_fixed, scales, zeros, G, codes, E,
+      err_sq);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+}
+
+gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, int64_t cols,
+                               int64_t ldw, const float* R, int bits, int group, int block,
+                               float* Wh, uint8_t* codes, float* scales, uint8_t* zeros,
+                               float* err_sq, void* ws, int32_t* info, cudaStream_t stream) {
+  (void)info;
+  float* E = static_cast<float*>(ws);
+  const int G = group > 0 ? static_cast<int>(cols / group) : 1;
+  const int64_t total = rows * cols;
+  const int cgrid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 8 * 148));
+  if (w_dtype == GPTQ_BF16)
+    convert_kernel<__nv_bfloat16><<<cgrid, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(W), ldw, Wh, rows, cols);
+  else
+    convert_kernel<float><<<cgrid, 256, 0, stream>>>(static_cast<const float*>(W), ldw, Wh, rows,
+                                                     cols);
+  count_launch();
+  if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
+  if (err_sq != nullptr && cudaMemsetAsync(err_sq, 0, rows * sizeof(float), stream) != cudaSuccess)
+    return GPTQ_ECUDA;
+  const unsigned pgrid = static_cast<unsigned>((rows + 7) / 8);
+  if (group <= 0) {
+    params_kernel<<<pgrid, 256, 0, stream>>>(Wh, rows, cols, 0, cols, bits, scales, zeros, 1, 0);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
+  }
+  for (int64_t b0 = 0; b0 < cols; b0 += block) {
+    const int nb = static_cast<int>(cols - b0 < block ? cols - b0 : block);
+    int mode = 0, gi = 0;
+    if (group > 0 && group % block == 0) {
+      gi = static_cast<int>(b0 / group);
+      if (b0 % group == 0) {
+        params_kernel<<<pgrid, 256, 0, stream>>>(Wh, rows, cols, b0, group, bits, scales, zeros, G,
+                                                 gi);
+        count_launch();
+        if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
+      }
+    } else if (group > 0) {
+      mode = 1;
+    }
+    gptq_status st;
+    switch (block) {
+      case 32:
+        st = launch_column_loop<32>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group, mode,
+                                    gi, scales, zeros, G, codes, E, err_sq, stream);
+        break;
+      case 64:
+        st = launch_column_loop<64>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group, mode,
+                                    gi, scales, zeros, G, codes, E, err_sq, stream);
+        break;
+      default:
+        st = launch_column_loop<128>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group,
+                                     mode, gi, scales, zeros, G, codes, E, err_sq, stream);
+        break;
+    }
+    if (st != GPTQ_OK) return st;
+    const int64_t b1 = b0 + nb;
+    if (b1 < cols) {
+      // S8: W[:, b1:] -= E * R[b0:b1, b1:]
+      GemmArgs g{E, block, 0, R + b0 * cols + b1, cols, 0, Wh + b1, cols, static_cast<int>(rows),
+                 static_cast<int>(cols - b1), nb, -1.f, 1.f, 0, 0, 0};
+      st = launch_gemm_f32(g, stream);
+      if (st != GPTQ_OK) return st;
+    }
+  }
+  return GPTQ_OK;
+}
+
+}  // namespace gptq

@@ -27,3 +27,12 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(scope="session")
+def built_lib():
+    """Path of libgptq_b200.so, building it in-tree with nvcc if it is missing."""
+    from post_weight_quantization_12_b200 import _lib, build
+    if not os.path.exists(_lib.LIB_PATH):
+        build.build()
+    return _lib.LIB_PATH

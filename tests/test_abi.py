@@ -1,0 +1,85 @@
+"""The C ABI library loads without a GPU, exports every entry point its header declares, and
+rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from post_weight_quantization_12_b200 import _lib
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include",
+                      "gptq.h")
+FAKE = ctypes.c_void_p(0x10000)   # never dereferenced: every call below fails validation first
+
+
+def declared_functions():
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    return sorted(set(re.findall(r"\b(gptq_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_path():
+    names = declared_functions()
+    for n in ("gptq_hessian_accumulate", "gptq_prepare_hinv", "gptq_quantize_layer",
+              "gptq_workspace_size", "gptq_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(built_lib):
+    lib = ctypes.CDLL(built_lib)
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) <= set(_lib.SIGNATURES)
+
+
+def test_status_strings_and_info_mapping(built_lib):
+    assert _lib.status_string(0) == "GPTQ_OK"
+    assert "EINVAL" in _lib.status_string(1)
+    assert _lib.info_status(0) == _lib.GPTQ_OK
+    assert _lib.info_status(7) == _lib.GPTQ_ENOTPD
+    assert _lib.info_status(-1) == _lib.GPTQ_ETIMEOUT
+    assert _lib.load().gptq_version().decode().count(".") == 2
+
+
+def test_workspace_sizes(built_lib):
+    q = _lib.workspace_size(_lib.GPTQ_WS_QUANTIZE, 4096, 4096, 128)
+    assert q >= 4096 * 128 * 4 and q % 256 == 0
+    p = _lib.workspace_size(_lib.GPTQ_WS_PREPARE, 0, 4096, 0)
+    assert p >= 4096 * 4096 * 4
+    assert _lib.workspace_size(_lib.GPTQ_WS_QUANTIZE, 10, 10, 48) == 0
+    assert _lib.workspace_size(99, 10, 10, 32) == 0
+
+
+@pytest.mark.parametrize("bits,group,block,cols,ldw", [
+    (1, -1, 128, 256, 256),      # bits below range
+    (9, -1, 128, 256, 256),      # bits above range
+    (4, 48, 32, 480, 480),       # group and block do not nest
+    (4, 128, 128, 200, 200),     # cols not a multiple of the group
+    (4, -1, 96, 256, 256),       # unsupported block
+    (4, 0, 128, 256, 256),       # group 0
+    (4, -1, 128, 256, 100),      # ldw < cols
+])
+def test_quantize_rejects_bad_arguments(built_lib, bits, group, block, cols, ldw):
+    lib = _lib.load()
+    st = lib.gptq_quantize_layer(FAKE, _lib.GPTQ_BF16, 64, cols, ldw, FAKE, bits, group, block,
+                                 FAKE, FAKE, FAKE, FAKE, None, FAKE, 1 << 30, FAKE, None)
+    assert st == _lib.GPTQ_EINVAL
+
+
+def test_other_entry_points_reject_bad_arguments(built_lib):
+    lib = _lib.load()
+    assert lib.gptq_hessian_accumulate(None, 128, FAKE, 0, 10, 128, FAKE, None) == _lib.GPTQ_EINVAL
+    assert lib.gptq_hessian_accumulate(FAKE, 128, FAKE, 0, 10, 64, FAKE, None) == _lib.GPTQ_EINVAL
+    # bf16 path needs 16-byte rows and base
+    assert lib.gptq_hessian_accumulate(FAKE, 12, FAKE, 0, 10, 12, FAKE, None) == _lib.GPTQ_EINVAL
+    assert lib.gptq_hessian_accumulate(FAKE, 128, FAKE, 0, 0, 128, FAKE, None) == _lib.GPTQ_OK
+    assert lib.gptq_prepare_hinv(FAKE, FAKE, 128, 0, 0.01, FAKE, 1 << 30, FAKE, None) == \
+        _lib.GPTQ_EINVAL
+    assert lib.gptq_prepare_hinv(FAKE, FAKE, 128, 10, -1.0, FAKE, 1 << 30, FAKE, None) == \
+        _lib.GPTQ_EINVAL
+    assert lib.gptq_prepare_hinv(FAKE, FAKE, 128, 10, 0.01, FAKE, 16, FAKE, None) == \
+        _lib.GPTQ_EWORKSPACE
+    st = lib.gptq_quantize_layer(FAKE, _lib.GPTQ_FP32, 64, 128, 128, FAKE, 4, -1, 32, FAKE, FAKE,
+                                 FAKE, FAKE, None, FAKE, 16, FAKE, None)
+    assert st == _lib.GPTQ_EWORKSPACE
+    assert lib.gptq_selftest_wait_timeout(FAKE, 0, None) == _lib.GPTQ_EINVAL
