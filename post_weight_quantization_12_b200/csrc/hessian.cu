@@ -30,6 +30,11 @@ constexpr int kStageBytes = 2 * kSlabBytes;          // A slab + B slab
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;
 constexpr int kThreads = 192;              // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 constexpr uint32_t kTmemCols = 512;
+// The tensor core adds each 16-deep product into the fp32 accumulator with a rounding that is
+// biased toward zero, so the relative error of a TMEM sum grows with the number of MMAs folded
+// into it (about 6e-8 per MMA measured on B200). Every kKbPerFlush stages (2048 tokens) the
+// chunk sum is added into S with IEEE fp32 adds and the accumulator restarts.
+constexpr int kKbPerFlush = 64;
 constexpr uint32_t kIdesc = make_idesc(/*bf16*/ 1, /*A MN-major*/ 1, /*B MN-major*/ 1, 128, 256);
 }  // namespace syrk
 
@@ -43,7 +48,7 @@ __device__ __forceinline__ void decode_lower(int st, int& I, int& J) {
 
 __global__ void __launch_bounds__(syrk::kThreads, 1)
 hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ S, int cols,
-                     int n_kblocks, int n_super, int32_t* info) {
+                     int n_kblocks, int kb_per_flush, int n_super, int32_t* info) {
   using namespace syrk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -120,28 +125,32 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
         int I, J;
         decode_lower(st, I, J);
         const bool diag = (I == J);
-        if (!mbar_wait_bounded(&acc_empty, aph ^ 1u, &abort_flag, info)) break;
-        tc_fence_after();
-        for (int kb = 0; kb < n_kblocks; ++kb) {
-          if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag, info)) goto mma_done_label;
+        for (int kc = 0; kc < n_kblocks; kc += kb_per_flush) {
+          // a fresh chunk sum in TMEM; the epilogue folds it into S with IEEE fp32 adds
+          if (!mbar_wait_bounded(&acc_empty, aph ^ 1u, &abort_flag, info)) goto mma_done_label;
           tc_fence_after();
-          const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
-          const uint32_t b_addr = diag ? a_addr : a_addr + kSlabBytes;
+          const int kc_end = min(n_kblocks, kc + kb_per_flush);
+          for (int kb = kc; kb < kc_end; ++kb) {
+            if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag, info)) goto mma_done_label;
+            tc_fence_after();
+            const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+            const uint32_t b_addr = diag ? a_addr : a_addr + kSlabBytes;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t bdesc = smem_desc(b_addr + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t bdesc = smem_desc(b_addr + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint64_t adesc =
-                  smem_desc(a_addr + 2 * h * kBoxBytes + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
-              tc_mma_f16(tmem + h * 256, adesc, bdesc, kIdesc, (kb | kk) != 0 ? 1u : 0u);
+              for (int h = 0; h < 2; ++h) {
+                const uint64_t adesc = smem_desc(a_addr + 2 * h * kBoxBytes + kk * 2048, kBoxBytes,
+                                                 1024, kSwizzle128B);
+                tc_mma_f16(tmem + h * 256, adesc, bdesc, kIdesc, (kb > kc || kk > 0) ? 1u : 0u);
+              }
             }
+            tc_commit(&empty_bar[s]);
+            if (++s == kStages) { s = 0; ph ^= 1u; }
           }
-          tc_commit(&empty_bar[s]);
-          if (++s == kStages) { s = 0; ph ^= 1u; }
+          tc_commit(&acc_full);
+          aph ^= 1u;
         }
-        tc_commit(&acc_full);
-        aph ^= 1u;
       }
     mma_done_label:
       tc_commit(&mma_done);
@@ -155,37 +164,40 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
     for (int st = blockIdx.x; st < n_super && !abort_flag; st += gridDim.x) {
       int I, J;
       decode_lower(st, I, J);
-      if (!mbar_wait_bounded(&acc_full, aph, &abort_flag, info)) break;
-      tc_fence_after();
+      for (int kc = 0; kc < n_kblocks; kc += kb_per_flush) {
+        if (!mbar_wait_bounded(&acc_full, aph, &abort_flag, info)) goto epilogue_done;
+        tc_fence_after();
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int i = I * 256 + h * 128 + r_in_half;
+        for (int h = 0; h < 2; ++h) {
+          const int i = I * 256 + h * 128 + r_in_half;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256 + c * 32, v);
-          tmem_wait_ld();
-          const int j0 = J * 256 + c * 32;
-          if (i < cols) {
-            float4* row = reinterpret_cast<float4*>(S + static_cast<size_t>(i) * cols + j0);
+          for (int c = 0; c < 8; ++c) {
+            uint32_t v[32];
+            tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256 + c * 32, v);
+            tmem_wait_ld();
+            const int j0 = J * 256 + c * 32;
+            if (i < cols) {
+              float4* row = reinterpret_cast<float4*>(S + static_cast<size_t>(i) * cols + j0);
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              if (j0 + 4 * t < cols) {
-                float4 o = row[t];
-                o.x += __uint_as_float(v[4 * t + 0]);
-                o.y += __uint_as_float(v[4 * t + 1]);
-                o.z += __uint_as_float(v[4 * t + 2]);
-                o.w += __uint_as_float(v[4 * t + 3]);
-                row[t] = o;
+              for (int t = 0; t < 8; ++t) {
+                if (j0 + 4 * t < cols) {
+                  float4 o = row[t];
+                  o.x += __uint_as_float(v[4 * t + 0]);
+                  o.y += __uint_as_float(v[4 * t + 1]);
+                  o.z += __uint_as_float(v[4 * t + 2]);
+                  o.w += __uint_as_float(v[4 * t + 3]);
+                  row[t] = o;
+                }
               }
             }
           }
         }
+        tc_fence_before();
+        mbar_arrive(&acc_empty);
+        aph ^= 1u;
       }
-      tc_fence_before();
-      mbar_arrive(&acc_empty);
-      aph ^= 1u;
     }
+  epilogue_done:;
   }
 
   tc_fence_before();
@@ -272,7 +284,7 @@ gptq_status launch_hessian_bf16(float* S, int64_t cols, const void* X, int64_t n
   if (n_kb > INT32_MAX / kBK) return GPTQ_EUNSUPPORTED;
   const int grid = n_super < num_sms() ? n_super : num_sms();
   hessian_syrk_bf16_tc<<<grid, kThreads, kSmemBytes, stream>>>(
-      tmap, S, static_cast<int>(cols), static_cast<int>(n_kb), n_super, info);
+      tmap, S, static_cast<int>(cols), static_cast<int>(n_kb), kKbPerFlush, n_super, info);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }
