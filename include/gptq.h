@@ -149,6 +149,32 @@ gptq_status gptq_quantize_layer(const void* W_dev, gptq_dtype w_dtype, int64_t r
                                 uint8_t* zeros_dev, float* err_sq_dev, void* ws_dev,
                                 size_t ws_bytes, int32_t* info_dev, void* stream);
 
+/*
+ * gptq_quantize_layer without a workspace argument, for callers that cannot allocate device
+ * memory (no counterpart on the pages: it packages the same S6-S8 computation differently).
+ *
+ * Who needs it: code whose host framework owns all device memory through its own pool, where a
+ * cudaMalloc of its own would fail or break the pool's accounting, and code that may not pay
+ * cudaMalloc's implicit device-wide synchronization. It computes exactly what gptq_quantize_layer
+ * computes, with the same arguments and outputs (the caller still passes all inputs and outputs),
+ * but keeps the error buffer E in a scratch array compiled into the library:
+ *   - size GPTQ_NOALLOC_SCRATCH_BYTES; every GPU that loads the library holds it until exit;
+ *   - calls needing more than that (rows * block * 4 bytes, rounded up to 256) return
+ *     GPTQ_EWORKSPACE without enqueueing anything; e.g. up to 8192 rows at block 128;
+ *   - the first call on each device looks up the array's device address (cudaGetSymbolAddress
+ *     with that device current); make that first call before any stream capture;
+ *   - all calls in the process share the one array per device and it keeps the last call's
+ *     contents (nothing in it needs to start at zero); calls whose work overlaps on the GPU, e.g.
+ *     on two streams at once, race on it -- serialize them.
+ * Errors: as gptq_quantize_layer, plus GPTQ_EWORKSPACE when the size limit is exceeded.
+ */
+#define GPTQ_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+gptq_status gptq_quantize_layer_noalloc(const void* W_dev, gptq_dtype w_dtype, int64_t rows,
+                                        int64_t cols, int64_t ldw, const float* R_dev, int bits,
+                                        int group, int block, float* W_hat_dev, uint8_t* codes_dev,
+                                        float* scales_dev, uint8_t* zeros_dev, float* err_sq_dev,
+                                        int32_t* info_dev, void* stream);
+
 /* Workspace bytes needed by one call (GPTQ_WS_PREPARE or GPTQ_WS_QUANTIZE); 0 for bad input. */
 size_t gptq_workspace_size(int which, int64_t rows, int64_t cols, int block);
 

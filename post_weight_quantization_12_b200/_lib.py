@@ -18,6 +18,7 @@ GPTQ_BF16, GPTQ_FP32 = 0, 1
 GPTQ_INFO_TIMEOUT = -1
 GPTQ_INFO_BAD_HESSIAN = -2
 GPTQ_WS_PREPARE, GPTQ_WS_QUANTIZE = 1, 2
+GPTQ_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 # name -> (restype, argtypes)
 _P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -30,6 +31,8 @@ SIGNATURES = {
     "gptq_info_status": (_I32, [ctypes.c_int32]),
     "gptq_status_string": (ctypes.c_char_p, [_I32]),
     "gptq_version": (ctypes.c_char_p, []),
+    "gptq_quantize_layer_noalloc": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _I32, _I32, _P,
+                                           _P, _P, _P, _P, _P, _P]),
     "gptq_kernel_launches": (ctypes.c_uint64, []),
     "gptq_selftest_wait_timeout": (_I32, [_P, _I32, _P]),
 }
@@ -139,3 +142,16 @@ def quantize_layer(W, R, bits, group, block, W_hat, codes, scales, zeros, err_sq
         int(block), _ptr(W_hat), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(err_sq), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(info), _stream(stream))
     _check(st, "gptq_quantize_layer")
+
+
+def quantize_layer_noalloc(W, R, bits, group, block, W_hat, codes, scales, zeros, err_sq, info,
+                           stream=None):
+    """As quantize_layer, but with the library's built-in scratch instead of a workspace (for
+    callers that cannot allocate device memory; limited to rows * block * 4 bytes of
+    GPTQ_NOALLOC_SCRATCH_BYTES; concurrent calls race on the shared scratch)."""
+    ldw = _row_major_ld(W, "W")
+    st = load().gptq_quantize_layer_noalloc(
+        _ptr(W), _dtype_code(W), W.shape[0], W.shape[1], ldw, _ptr(R), int(bits), int(group),
+        int(block), _ptr(W_hat), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(err_sq), _ptr(info),
+        _stream(stream))
+    _check(st, "gptq_quantize_layer_noalloc")

@@ -1,0 +1,78 @@
+"""gptq_quantize_layer_noalloc: the column loop for callers that cannot allocate device memory
+(for example code whose framework owns every device allocation through its own pool, or code that
+cannot afford cudaMalloc's implicit synchronization). It keeps its error buffer in scratch built
+into the library instead of a caller workspace, so its results must equal those of
+gptq_quantize_layer on the same inputs -- checked here on two calls in a row, the second with
+other shapes, so that whatever the first call left in the shared scratch cannot leak into it.
+
+This file is collected last on purpose and also passes when run alone in a fresh process.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from post_weight_quantization_12_b200 import _lib, synth
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _problem(rows, cols, seed):
+    spec = synth.scaled_spec(synth.ATTN, rows, cols, 4 * cols)
+    W = synth.weights_np(spec, seed)
+    H = oracle.hessian(synth.inputs_np(spec, seed))
+    R = oracle.inverse_hessian_factor(H)["R"].astype(np.float32)
+    return (torch.from_numpy(W).to(DEV).to(torch.bfloat16), torch.from_numpy(R).to(DEV))
+
+
+def _outputs(rows, cols, group):
+    G = 1 if group <= 0 else cols // group
+    return dict(W_hat=torch.empty(rows, cols, device=DEV),
+                codes=torch.empty(rows, cols, dtype=torch.uint8, device=DEV),
+                scales=torch.empty(rows, G, device=DEV),
+                zeros=torch.empty(rows, G, dtype=torch.uint8, device=DEV),
+                err_sq=torch.empty(rows, device=DEV))
+
+
+def _run(W, R, bits, group, block, noalloc):
+    rows, cols = W.shape
+    out = _outputs(rows, cols, group)
+    info = torch.zeros(1, dtype=torch.int32, device=DEV)
+    if noalloc:
+        _lib.quantize_layer_noalloc(W, R, bits, group, block, out["W_hat"], out["codes"],
+                                    out["scales"], out["zeros"], out["err_sq"], info)
+    else:
+        ws = torch.empty(_lib.workspace_size(_lib.GPTQ_WS_QUANTIZE, rows, cols, block),
+                         dtype=torch.uint8, device=DEV)
+        _lib.quantize_layer(W, R, bits, group, block, out["W_hat"], out["codes"], out["scales"],
+                            out["zeros"], out["err_sq"], ws, info)
+    torch.cuda.synchronize()
+    assert info.item() == 0
+    return {k: v.cpu().numpy() for k, v in out.items()}
+
+
+@pytest.mark.parametrize("call", [
+    (1024, 1024, 4, 128, 128),   # first call: 1024 rows x block 128 (512 KB of scratch)
+    (300, 640, 3, -1, 64),       # second call: other shapes, per-row grid, ragged row count
+])
+def test_noalloc_matches_workspace_entry_point(call):
+    rows, cols, bits, group, block = call
+    W, R = _problem(rows, cols, seed=rows)
+    ref = _run(W, R, bits, group, block, noalloc=False)
+    got = _run(W, R, bits, group, block, noalloc=True)
+    # The same deterministic kernels run on the same inputs, so the results must be identical,
+    # which is stricter than the parity tolerance (>= 99.5 % of codes, 1 % layer error).
+    for k in ("codes", "scales", "zeros", "W_hat", "err_sq"):
+        np.testing.assert_array_equal(got[k], ref[k], err_msg=k)
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch():
+    lib = _lib.load()
+    fake = ctypes.c_void_p(0x10000)      # never touched: the size check comes first
+    rows = _lib.GPTQ_NOALLOC_SCRATCH_BYTES // (128 * 4) + 1
+    st = lib.gptq_quantize_layer_noalloc(fake, _lib.GPTQ_BF16, rows, 128, 128, fake, 4, -1, 128,
+                                         fake, fake, fake, fake, None, fake, None)
+    assert st == _lib.GPTQ_EWORKSPACE
