@@ -100,7 +100,10 @@ gptq_status gptq_hessian_accumulate(float* S_dev, int64_t cols, const void* X_de
  *   ws_dev     device workspace of at least gptq_workspace_size(GPTQ_WS_PREPARE, 0, cols, 0)
  *              bytes, 256-byte aligned; contents on entry do not matter.
  *   info_dev   status word: pivot codes (see GPTQ_INFO_*), GPTQ_INFO_BAD_HESSIAN.
- * Errors: GPTQ_EINVAL (null pointers, cols <= 0, n_total <= 0, damp_rel < 0), GPTQ_EWORKSPACE.
+ * Requirements: cols % 4 == 0; S_H_dev and R_dev 16-byte aligned (the matrix products run on
+ * the tensor cores through TMA, whose rows must start on 16-byte boundaries).
+ * Errors: GPTQ_EINVAL (null pointers, cols <= 0 or not a multiple of 4, misaligned buffers,
+ * n_total <= 0, damp_rel < 0), GPTQ_EWORKSPACE.
  */
 gptq_status gptq_prepare_hinv(float* S_H_dev, float* R_dev, int64_t cols, int64_t n_total,
                               float damp_rel, void* ws_dev, size_t ws_bytes, int32_t* info_dev,
@@ -141,7 +144,9 @@ gptq_status gptq_prepare_hinv(float* S_H_dev, float* R_dev, int64_t cols, int64_
  *   ws_dev     device workspace of gptq_workspace_size(GPTQ_WS_QUANTIZE, rows, cols, block)
  *              bytes, 256-byte aligned.
  *   info_dev   status word.
- * Errors: GPTQ_EINVAL (shapes, bits, group/block rules, null pointers), GPTQ_EWORKSPACE.
+ * Requirements: cols % 4 == 0; R_dev and W_hat_dev 16-byte aligned.
+ * Errors: GPTQ_EINVAL (shapes, bits, group/block rules, alignment, null pointers),
+ * GPTQ_EWORKSPACE.
  */
 gptq_status gptq_quantize_layer(const void* W_dev, gptq_dtype w_dtype, int64_t rows, int64_t cols,
                                 int64_t ldw, const float* R_dev, int bits, int group, int block,
@@ -158,9 +163,12 @@ gptq_status gptq_quantize_layer(const void* W_dev, gptq_dtype w_dtype, int64_t r
  * cudaMalloc's implicit device-wide synchronization. It computes exactly what gptq_quantize_layer
  * computes, with the same arguments and outputs (the caller still passes all inputs and outputs),
  * but keeps the error buffer E in a scratch array compiled into the library:
- *   - size GPTQ_NOALLOC_SCRATCH_BYTES; every GPU that loads the library holds it until exit;
- *   - calls needing more than that (rows * block * 4 bytes, rounded up to 256) return
- *     GPTQ_EWORKSPACE without enqueueing anything; e.g. up to 8192 rows at block 128;
+ *   - size GPTQ_NOALLOC_SCRATCH_BYTES (16 MiB); every GPU that loads the library holds it
+ *     until exit;
+ *   - a call needing more than that, i.e. gptq_workspace_size(GPTQ_WS_QUANTIZE, rows, cols,
+ *     block) bytes (2 * rows * block * 4 + 2 * block * cols * 4, each part rounded up to 256),
+ *     returns GPTQ_EWORKSPACE without enqueueing anything; at block 128 a layer of up to
+ *     8192 x 8192 fits;
  *   - the first call on each device looks up the array's device address (cudaGetSymbolAddress
  *     with that device current); make that first call before any stream capture;
  *   - all calls in the process share the one array per device and it keeps the last call's
@@ -168,7 +176,7 @@ gptq_status gptq_quantize_layer(const void* W_dev, gptq_dtype w_dtype, int64_t r
  *     on two streams at once, race on it -- serialize them.
  * Errors: as gptq_quantize_layer, plus GPTQ_EWORKSPACE when the size limit is exceeded.
  */
-#define GPTQ_NOALLOC_SCRATCH_BYTES (4u * 1024u * 1024u)
+#define GPTQ_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 gptq_status gptq_quantize_layer_noalloc(const void* W_dev, gptq_dtype w_dtype, int64_t rows,
                                         int64_t cols, int64_t ldw, const float* R_dev, int bits,
                                         int group, int block, float* W_hat_dev, uint8_t* codes_dev,
@@ -196,6 +204,24 @@ uint64_t gptq_kernel_launches(void);
  * leaving the context usable. Lets callers check that a lost wait ends as a status, not a hang.
  */
 gptq_status gptq_selftest_wait_timeout(int32_t* info_dev, int limit_ms, void* stream);
+
+/*
+ * Self-test of the tensor-core matrix product every S3-S5 and S8 step runs on (no counterpart on
+ * the pages). Computes, in the 3xTF32 scheme (operands split into tf32 big/small parts; the
+ * small*small term is dropped):
+ *     C[m][n] = alpha * sum_{k = klo}^{K-1} opA[m][k] * opB[k][n] + beta * C[m][n]
+ *   opA[m][k] = a_mn ? A[k * lda + m] : A[m * lda + k];  opB[k][n] = b_mn ? B[k * ldb + n]
+ *   : B[n * ldb + k]; with `lower`, 128 x 128 tiles of C above the diagonal are left untouched;
+ *   klo = max(0, tile row start if klo_from_m, tile column start if klo_from_n).
+ * C_big / C_small (may be NULL) receive the tf32 split of the result with ld ldc.
+ * ws: at least 2 * (rows_A * lda + rows_B * ldb) * 4 bytes + 1024, where rows_A = a_mn ? K : M
+ * and rows_B = b_mn ? K : N. Requirements: lda, ldb, ldc multiples of 4; 16-byte aligned buffers.
+ */
+gptq_status gptq_selftest_gemm(const float* A_dev, int64_t lda, int a_mn, const float* B_dev,
+                               int64_t ldb, int b_mn, float* C_dev, int64_t ldc, int M, int N,
+                               int K, float alpha, float beta, int lower, int klo_from_m,
+                               int klo_from_n, float* C_big_dev, float* C_small_dev, void* ws_dev,
+                               size_t ws_bytes, int32_t* info_dev, void* stream);
 
 /* Library version, "major.minor.patch". */
 const char* gptq_version(void);

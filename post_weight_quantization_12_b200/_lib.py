@@ -18,7 +18,7 @@ GPTQ_BF16, GPTQ_FP32 = 0, 1
 GPTQ_INFO_TIMEOUT = -1
 GPTQ_INFO_BAD_HESSIAN = -2
 GPTQ_WS_PREPARE, GPTQ_WS_QUANTIZE = 1, 2
-GPTQ_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
+GPTQ_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 # name -> (restype, argtypes)
 _P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -34,6 +34,8 @@ SIGNATURES = {
     "gptq_quantize_layer_noalloc": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _I32, _I32, _P,
                                            _P, _P, _P, _P, _P, _P]),
     "gptq_kernel_launches": (ctypes.c_uint64, []),
+    "gptq_selftest_gemm": (_I32, [_P, _I64, _I32, _P, _I64, _I32, _P, _I64, _I32, _I32, _I32,
+                                  _F, _F, _I32, _I32, _I32, _P, _P, _P, _SZ, _P, _P]),
     "gptq_selftest_wait_timeout": (_I32, [_P, _I32, _P]),
 }
 
@@ -147,11 +149,27 @@ def quantize_layer(W, R, bits, group, block, W_hat, codes, scales, zeros, err_sq
 def quantize_layer_noalloc(W, R, bits, group, block, W_hat, codes, scales, zeros, err_sq, info,
                            stream=None):
     """As quantize_layer, but with the library's built-in scratch instead of a workspace (for
-    callers that cannot allocate device memory; limited to rows * block * 4 bytes of
-    GPTQ_NOALLOC_SCRATCH_BYTES; concurrent calls race on the shared scratch)."""
+    callers that cannot allocate device memory; limited to layers whose quantize workspace fits
+    in GPTQ_NOALLOC_SCRATCH_BYTES; concurrent calls race on the shared scratch)."""
     ldw = _row_major_ld(W, "W")
     st = load().gptq_quantize_layer_noalloc(
         _ptr(W), _dtype_code(W), W.shape[0], W.shape[1], ldw, _ptr(R), int(bits), int(group),
         int(block), _ptr(W_hat), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(err_sq), _ptr(info),
         _stream(stream))
     _check(st, "gptq_quantize_layer_noalloc")
+
+
+def selftest_gemm(A, a_mn, B, b_mn, C, M, N, K, alpha=1.0, beta=0.0, lower=False,
+                  klo_from_m=False, klo_from_n=False, C_big=None, C_small=None, info=None,
+                  stream=None):
+    """The library's tensor-core (3xTF32) matrix product on fp32 device tensors (self-test)."""
+    import torch
+    lda, ldb = _row_major_ld(A, "A"), _row_major_ld(B, "B")
+    ldc = _row_major_ld(C, "C") if C is not None else (C_big.stride(0) if C_big is not None else 4)
+    ws = torch.empty(2 * (A.shape[0] * lda + B.shape[0] * ldb) * 4 + 2048, dtype=torch.uint8,
+                     device=A.device)
+    st = load().gptq_selftest_gemm(_ptr(A), lda, int(a_mn), _ptr(B), ldb, int(b_mn), _ptr(C), ldc,
+                                   int(M), int(N), int(K), float(alpha), float(beta), int(lower),
+                                   int(klo_from_m), int(klo_from_n), _ptr(C_big), _ptr(C_small),
+                                   _ptr(ws), ws.numel(), _ptr(info), _stream(stream))
+    _check(st, "gptq_selftest_gemm")

@@ -108,6 +108,7 @@ gptq_status gptq_prepare_hinv(float* S_H_dev, float* R_dev, int64_t cols, int64_
                               float damp_rel, void* ws_dev, size_t ws_bytes, int32_t* info_dev,
                               void* stream) {
   if (S_H_dev == nullptr || R_dev == nullptr || cols <= 0 || n_total <= 0) return GPTQ_EINVAL;
+  if (cols % 4 != 0 || !aligned(S_H_dev, 16) || !aligned(R_dev, 16)) return GPTQ_EINVAL;
   if (!(damp_rel >= 0.f) || !(damp_rel < 1e30f)) return GPTQ_EINVAL;
   if (cols > 65536) return GPTQ_EUNSUPPORTED;
   if (ws_dev == nullptr || ws_bytes < prepare_workspace_bytes(cols) || !aligned(ws_dev, 256))
@@ -125,6 +126,7 @@ gptq_status gptq_quantize_layer(const void* W_dev, gptq_dtype w_dtype, int64_t r
       scales_dev == nullptr || zeros_dev == nullptr)
     return GPTQ_EINVAL;
   if (rows <= 0 || cols <= 0 || ldw < cols) return GPTQ_EINVAL;
+  if (cols % 4 != 0 || !aligned(R_dev, 16) || !aligned(W_hat_dev, 16)) return GPTQ_EINVAL;
   if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_FP32) return GPTQ_EINVAL;
   if (bits < 2 || bits > 8) return GPTQ_EINVAL;
   if (block != 32 && block != 64 && block != 128) return GPTQ_EINVAL;
@@ -180,6 +182,37 @@ gptq_status gptq_selftest_wait_timeout(int32_t* info_dev, int limit_ms, void* st
       info_dev, static_cast<uint64_t>(limit_ms) * 1000000ull);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+}
+
+gptq_status gptq_selftest_gemm(const float* A_dev, int64_t lda, int a_mn, const float* B_dev,
+                               int64_t ldb, int b_mn, float* C_dev, int64_t ldc, int M, int N,
+                               int K, float alpha, float beta, int lower, int klo_from_m,
+                               int klo_from_n, float* C_big_dev, float* C_small_dev, void* ws_dev,
+                               size_t ws_bytes, int32_t* info_dev, void* stream) {
+  if (A_dev == nullptr || B_dev == nullptr || ws_dev == nullptr || M <= 0 || N <= 0 || K < 0)
+    return GPTQ_EINVAL;
+  if (lda % 4 || ldb % 4 || ldc % 4 || (C_big_dev != nullptr) != (C_small_dev != nullptr))
+    return GPTQ_EINVAL;
+  if ((C_dev == nullptr && beta != 0.f) || !aligned(ws_dev, 256)) return GPTQ_EINVAL;
+  const int64_t ra = a_mn ? K : M, ca = a_mn ? M : K;
+  const int64_t rb = b_mn ? K : N, cb = b_mn ? N : K;
+  if (lda < ca || ldb < cb || (C_dev != nullptr && ldc < N)) return GPTQ_EINVAL;
+  const size_t a_bytes = align_up(static_cast<size_t>(ra) * lda * 4, 256);
+  const size_t b_bytes = align_up(static_cast<size_t>(rb) * ldb * 4, 256);
+  if (ws_bytes < 2 * a_bytes + 2 * b_bytes) return GPTQ_EWORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws_dev);
+  float* Ab = reinterpret_cast<float*>(w);
+  float* As = reinterpret_cast<float*>(w + a_bytes);
+  float* Bb = reinterpret_cast<float*>(w + 2 * a_bytes);
+  float* Bs = reinterpret_cast<float*>(w + 2 * a_bytes + b_bytes);
+  gptq_status st = launch_split_tf32(A_dev, lda, ra, ca, Ab, As, lda, s);
+  if (st != GPTQ_OK) return st;
+  if ((st = launch_split_tf32(B_dev, ldb, rb, cb, Bb, Bs, ldb, s)) != GPTQ_OK) return st;
+  TcGemmArgs g{Ab, As, Bb, Bs, lda, ldb, a_mn ? 1 : 0, b_mn ? 1 : 0, M, N, K, alpha, beta,
+               lower ? 1 : 0, klo_from_m ? 1 : 0, klo_from_n ? 1 : 0, C_dev, ldc, C_big_dev,
+               C_small_dev, ldc, info_dev};
+  return launch_gemm_tc(g, s);
 }
 
 const char* gptq_version(void) { return "0.1.0"; }

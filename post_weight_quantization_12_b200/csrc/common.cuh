@@ -184,6 +184,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes
   return d;
 }
 constexpr uint32_t kSwizzle128B = 2;
+constexpr uint32_t kSwizzle128B32BAtom = 1;  // 128-byte swizzle, 32-byte atoms (MN-major 32-bit)
 
 // Instruction descriptor for kind::f16 / kind::tf32 with fp32 accumulation.
 //   fmt: 0 = f16, 1 = bf16, 2 = tf32; a_mn/b_mn: operand is MN-major (1) or K-major (0).

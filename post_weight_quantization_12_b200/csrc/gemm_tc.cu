@@ -1,0 +1,340 @@
+// fp32-accurate matrix products on the tcgen05 tensor cores ("3xTF32").
+//
+// Every operand x is stored twice: x_big = x rounded to tf32 (10 explicit mantissa bits) and
+// x_small = x - x_big (exact in fp32). The product is a_big*b_big + (a_big*b_small + a_small*b_big);
+// the dropped a_small*b_small term and the tf32 truncation of the small parts leave a relative
+// error near 2^-21 per product, close to fp32.
+//
+// The tensor core adds each MMA's result into its fp32 accumulator with a rounding biased toward
+// zero, so long sums drift. The kernel therefore keeps two short-lived TMEM accumulators (the
+// big*big term and the two correction terms) per chunk of kChunkStages k-stages and folds each
+// chunk into a per-thread fp32 register accumulator with ordinary IEEE adds; the chunk buffers are
+// double-buffered so the MMAs never wait for the fold.
+//
+// One CTA per 128 x 128 output tile: warp 0 issues TMA loads (128-byte swizzle, either operand
+// K-major or MN-major), warp 1 issues the MMAs, warps 2-5 fold and write the tile:
+//   C = alpha * acc + beta * C    (C may be null), and optionally the tf32 split of the result.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gptq {
+
+namespace tg {
+constexpr int BM = 128, BN = 128, BK = 32;
+constexpr int kStages = 3;
+constexpr int kChunkStages = 8;                 // k-stages (256 k) per TMEM chunk sum
+constexpr int kOpBytes = BM * BK * 4;           // 16 KB per operand part per stage
+constexpr int kStageBytes = 4 * kOpBytes;       // A_big, A_small, B_big, B_small
+constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;             // 2 buffers x (main 128 + corr 128)
+}  // namespace tg
+
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+struct TcGemmParams {
+  int M, N, K;
+  int a_mn, b_mn;          // operand is MN-major (1) or K-major (0)
+  float alpha, beta;
+  int lower, klo_from_m, klo_from_n;
+  float* C;                // may be null
+  int64_t ldc;
+  float* Cbig;             // may be null: tf32 split of the result
+  float* Csmall;
+  int64_t ld_split;
+  int tiles_n;
+  int vec4;                // C / split rows are 16-byte aligned
+};
+
+__global__ void __launch_bounds__(tg::kThreads, 1)
+gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ CUtensorMap tAs,
+               const __grid_constant__ CUtensorMap tBb, const __grid_constant__ CUtensorMap tBs,
+               TcGemmParams p, int32_t* info) {
+  using namespace tg;
+  const int tm = blockIdx.x / p.tiles_n, tn = blockIdx.x % p.tiles_n;
+  const int m0 = tm * BM, n0 = tn * BN;
+  if (p.lower && n0 > m0 + BM - 1) return;  // tile entirely above the diagonal
+  int klo = 0;
+  if (p.klo_from_m) klo = max(klo, m0);
+  if (p.klo_from_n) klo = max(klo, n0);
+  const int nk = p.K > klo ? (p.K - klo + BK - 1) / BK : 0;
+  const int n_chunks = (nk + kChunkStages - 1) / kChunkStages;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    if (lane == 0 && nk > 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag, info)) break;
+        uint8_t* st = smem + s * kStageBytes;
+        const int k0 = klo + kb * BK;
+        mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
+        // A parts at st + 0 / kOpBytes, B parts at st + 2 / 3 * kOpBytes
+        if (p.a_mn) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            tma_load_2d(st + q * 4096, &tAb, &full_bar[s], m0 + 32 * q, k0);
+            tma_load_2d(st + kOpBytes + q * 4096, &tAs, &full_bar[s], m0 + 32 * q, k0);
+          }
+        } else {
+          tma_load_2d(st, &tAb, &full_bar[s], k0, m0);
+          tma_load_2d(st + kOpBytes, &tAs, &full_bar[s], k0, m0);
+        }
+        if (p.b_mn) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            tma_load_2d(st + 2 * kOpBytes + q * 4096, &tBb, &full_bar[s], n0 + 32 * q, k0);
+            tma_load_2d(st + 3 * kOpBytes + q * 4096, &tBs, &full_bar[s], n0 + 32 * q, k0);
+          }
+        } else {
+          tma_load_2d(st + 2 * kOpBytes, &tBb, &full_bar[s], k0, n0);
+          tma_load_2d(st + 3 * kOpBytes, &tBs, &full_bar[s], k0, n0);
+        }
+        ++issued;
+        if (++s == kStages) { s = 0; ph ^= 1u; }
+      }
+      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+        mbar_drain_bounded(&full_bar[i % kStages], static_cast<uint32_t>((i / kStages) & 1));
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nk > 0) {
+      const uint32_t idesc = make_idesc(/*tf32*/ 2, p.a_mn, p.b_mn, BM, BN);
+      // K-major (128-byte swizzle): rows of 128 B in 8-row atoms; a K step of 8 tf32 is +32 B
+      // inside the row. MN-major 32-bit operands must use the 128-byte swizzle with 32-byte atoms
+      // (layout type 1): 128-byte rows in 4-row groups (SBO 512 B), 32-element MN chunks 4 KB
+      // apart (LBO), a K step of 8 rows is +1024 B.
+      const uint32_t a_lbo = p.a_mn ? 4096u : 16u, b_lbo = p.b_mn ? 4096u : 16u;
+      const uint32_t a_sbo = p.a_mn ? 512u : 1024u, b_sbo = p.b_mn ? 512u : 1024u;
+      const uint32_t a_lay = p.a_mn ? kSwizzle128B32BAtom : kSwizzle128B;
+      const uint32_t b_lay = p.b_mn ? kSwizzle128B32BAtom : kSwizzle128B;
+      const uint32_t a_step = p.a_mn ? 1024u : 32u, b_step = p.b_mn ? 1024u : 32u;
+      int s = 0;
+      uint32_t ph = 0;
+      int kb = 0;
+      for (int c = 0; c < n_chunks; ++c) {
+        const int buf = c & 1;
+        if (!mbar_wait_bounded(&acc_empty[buf], ((c >> 1) & 1) ^ 1u, &abort_flag, info)) break;
+        tc_fence_after();
+        const uint32_t t_main = tmem + buf * 256, t_corr = t_main + 128;
+        const int kb_end = min(nk, kb + kChunkStages);
+        bool first = true;
+        bool ok = true;
+        for (; kb < kb_end; ++kb) {
+          if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag, info)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t base = smem_u32(smem + s * kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 8; ++kk) {
+            const uint64_t ab = smem_desc(base + kk * a_step, a_lbo, a_sbo, a_lay);
+            const uint64_t as = smem_desc(base + kOpBytes + kk * a_step, a_lbo, a_sbo, a_lay);
+            const uint64_t bb = smem_desc(base + 2 * kOpBytes + kk * b_step, b_lbo, b_sbo, b_lay);
+            const uint64_t bs = smem_desc(base + 3 * kOpBytes + kk * b_step, b_lbo, b_sbo, b_lay);
+            tc_mma_tf32(t_corr, ab, bs, idesc, first ? 0u : 1u);
+            tc_mma_tf32(t_corr, as, bb, idesc, 1u);
+            tc_mma_tf32(t_main, ab, bb, idesc, first ? 0u : 1u);
+            first = false;
+          }
+          tc_commit(&empty_bar[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(&acc_full[buf]);
+      }
+      tc_commit(&mma_done);
+      mbar_drain_bounded(&mma_done, 0);
+    }
+  } else {
+    // ---------------- epilogue: fold chunks into registers, then write ----------------
+    const int q = warp & 3;
+    const int row = m0 + q * 32 + lane;
+    float acc[BN];
+#pragma unroll
+    for (int j = 0; j < BN; ++j) acc[j] = 0.f;
+    bool ok = true;
+    for (int c = 0; c < n_chunks; ++c) {
+      const int buf = c & 1;
+      if (!mbar_wait_bounded(&acc_full[buf], (c >> 1) & 1, &abort_flag, info)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t t_main = tmem + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t vm[32], vc[32];
+        tmem_ld_32x32b_x32(t_main + cc * 32, vm);
+        tmem_ld_32x32b_x32(t_main + 128 + cc * 32, vc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+          acc[cc * 32 + t] += __uint_as_float(vm[t]) + __uint_as_float(vc[t]);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+    }
+    if (ok && row < p.M) {
+      float* crow = p.C ? p.C + static_cast<int64_t>(row) * p.ldc + n0 : nullptr;
+      float* brow = p.Cbig ? p.Cbig + static_cast<int64_t>(row) * p.ld_split + n0 : nullptr;
+      float* srow = p.Cbig ? p.Csmall + static_cast<int64_t>(row) * p.ld_split + n0 : nullptr;
+      const int ncol = min(BN, p.N - n0);
+      if (p.vec4 && ncol == BN) {
+#pragma unroll
+        for (int j = 0; j < BN; j += 4) {
+          float4 v = make_float4(p.alpha * acc[j], p.alpha * acc[j + 1], p.alpha * acc[j + 2],
+                                 p.alpha * acc[j + 3]);
+          if (p.beta != 0.f) {
+            const float4 o = *reinterpret_cast<const float4*>(crow + j);
+            v.x = fmaf(p.beta, o.x, v.x); v.y = fmaf(p.beta, o.y, v.y);
+            v.z = fmaf(p.beta, o.z, v.z); v.w = fmaf(p.beta, o.w, v.w);
+          }
+          if (crow) *reinterpret_cast<float4*>(crow + j) = v;
+          if (brow) {
+            const float4 b = make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z),
+                                         tf32_round(v.w));
+            *reinterpret_cast<float4*>(brow + j) = b;
+            *reinterpret_cast<float4*>(srow + j) =
+                make_float4(v.x - b.x, v.y - b.y, v.z - b.z, v.w - b.w);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < BN; ++j) {
+          if (j < ncol) {
+            float v = p.alpha * acc[j];
+            if (p.beta != 0.f) v = fmaf(p.beta, crow[j], v);
+            if (crow) crow[j] = v;
+            if (brow) {
+              const float b = tf32_round(v);
+              brow[j] = b;
+              srow[j] = v - b;
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// x -> (tf32(x), x - tf32(x)) for a rows x cols block (row-major, leading dims in elements).
+__global__ void split_tf32_kernel(const float* __restrict__ X, int64_t ldx, int64_t rows,
+                                  int64_t cols, float* __restrict__ big, float* __restrict__ small,
+                                  int64_t ldo) {
+  const int64_t total = rows * cols;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = e / cols, c = e - r * cols;
+    const float x = X[r * ldx + c];
+    const float b = tf32_round(x);
+    big[r * ldo + c] = b;
+    small[r * ldo + c] = x - b;
+  }
+}
+
+gptq_status launch_split_tf32(const float* X, int64_t ldx, int64_t rows, int64_t cols, float* big,
+                              float* small, int64_t ldo, cudaStream_t stream) {
+  if (rows <= 0 || cols <= 0) return GPTQ_OK;
+  const int64_t total = rows * cols;
+  const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 16 * 148));
+  split_tf32_kernel<<<grid, 256, 0, stream>>>(X, ldx, rows, cols, big, small, ldo);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+}
+
+static gptq_status operand_map(CUtensorMap* m, const float* base, int64_t ld, int mn_major,
+                               int64_t mn_extent, int64_t k_extent) {
+  // K-major: dims {K, MN}, box {32, 128}, 128-byte swizzle; MN-major: dims {MN, K}, box {32, 32},
+  // 128-byte swizzle with 32-byte atoms (the only MN-major layout tcgen05 takes for tf32).
+  if (mn_major)
+    return encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, 4, mn_extent, k_extent, ld,
+                          32, 32, CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B);
+  return encode_tmap_2d(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, base, 4, k_extent, mn_extent, ld, 32,
+                        128, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
+  using namespace tg;
+  if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
+  if (!al16(g.Ab) || !al16(g.As) || !al16(g.Bb) || !al16(g.Bs) || g.lda % 4 || g.ldb % 4)
+    return GPTQ_EINVAL;
+  const int K = g.K > 0 ? g.K : 1;  // an empty K still needs valid maps
+  CUtensorMap tAb, tAs, tBb, tBs;
+  gptq_status st;
+  if ((st = operand_map(&tAb, g.Ab, g.lda, g.a_mn, g.M, K)) != GPTQ_OK) return st;
+  if ((st = operand_map(&tAs, g.As, g.lda, g.a_mn, g.M, K)) != GPTQ_OK) return st;
+  if ((st = operand_map(&tBb, g.Bb, g.ldb, g.b_mn, g.N, K)) != GPTQ_OK) return st;
+  if ((st = operand_map(&tBs, g.Bs, g.ldb, g.b_mn, g.N, K)) != GPTQ_OK) return st;
+  static bool attr_done = false;
+  if (!attr_done) {
+    if (cudaFuncSetAttribute(gemm_tf32x3_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kSmemBytes) != cudaSuccess)
+      return GPTQ_ECUDA;
+    attr_done = true;
+  }
+  TcGemmParams p;
+  p.M = g.M; p.N = g.N; p.K = g.K;
+  p.a_mn = g.a_mn; p.b_mn = g.b_mn;
+  p.alpha = g.alpha; p.beta = g.beta;
+  p.lower = g.lower; p.klo_from_m = g.klo_from_m; p.klo_from_n = g.klo_from_n;
+  p.C = g.C; p.ldc = g.ldc;
+  p.Cbig = g.Cbig; p.Csmall = g.Csmall; p.ld_split = g.ld_split;
+  p.tiles_n = (g.N + BN - 1) / BN;
+  const int tiles_m = (g.M + BM - 1) / BM;
+  p.vec4 = ((g.C == nullptr || (al16(g.C) && g.ldc % 4 == 0)) &&
+            (g.Cbig == nullptr || (al16(g.Cbig) && al16(g.Csmall) && g.ld_split % 4 == 0)))
+               ? 1 : 0;
+  const int64_t grid = static_cast<int64_t>(tiles_m) * p.tiles_n;
+  if (grid > 0x7fffffff) return GPTQ_EUNSUPPORTED;
+  gemm_tf32x3_tc<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(tAb, tAs, tBb, tBs,
+                                                                                 p, g.info);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+}
+
+}  // namespace gptq

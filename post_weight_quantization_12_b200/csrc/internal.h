@@ -24,27 +24,38 @@ gptq_status launch_hessian_bf16(float* S, int64_t cols, const void* X, int64_t n
 gptq_status launch_hessian_f32(float* S, int64_t cols, const float* X, int64_t n_tokens,
                                int64_t ldx, cudaStream_t stream);
 
-// General fp32 matrix product on one tile grid:
-//   C[m][n] = beta * C[m][n] + alpha * sum_{k = klo(m0, n0)}^{K-1} opA[m][k] * opB[k][n]
-// opA[m][k] = transA ? A[k * lda + m] : A[m * lda + k]; opB likewise with B. With `lower`, output
-// tiles lying entirely above the diagonal m == n are skipped. klo = max(0, m0 if klo_from_m,
-// n0 if klo_from_n) where m0/n0 are the tile's first row/column (skips known-zero triangles).
-struct GemmArgs {
-  const float* A;
-  int64_t lda;
-  int transA;
-  const float* B;
-  int64_t ldb;
-  int transB;
-  float* C;
-  int64_t ldc;
+// fp32-accurate matrix product on the tensor cores (3xTF32, see gemm_tc.cu):
+//   C[m][n] = alpha * sum_{k = klo}^{K-1} opA[m][k] * opB[k][n] + beta * C[m][n]
+// Each operand comes as its tf32 split (x_big, x_small), both with the same layout:
+//   opA[m][k] = a_mn ? A[k * lda + m] : A[m * lda + k]
+//   opB[k][n] = b_mn ? B[k * ldb + n] : B[n * ldb + k]
+// With `lower`, 128 x 128 output tiles entirely above the diagonal m == n are skipped.
+// klo = max(0, m0 if klo_from_m, n0 if klo_from_n) for the tile's first row m0 / column n0, to
+// skip known-zero triangles (m0, n0 are multiples of 128). C may be null (then beta must be 0);
+// if Cbig is set, the tf32 split of the result is also written there (ld_split).
+// Requirements: operand bases 16-byte aligned, lda % 4 == 0, ldb % 4 == 0.
+struct TcGemmArgs {
+  const float* Ab;
+  const float* As;
+  const float* Bb;
+  const float* Bs;
+  int64_t lda, ldb;
+  int a_mn, b_mn;
   int M, N, K;
   float alpha, beta;
-  int lower;
-  int klo_from_m;
-  int klo_from_n;
+  int lower, klo_from_m, klo_from_n;
+  float* C;
+  int64_t ldc;
+  float* Cbig;
+  float* Csmall;
+  int64_t ld_split;
+  int32_t* info;
 };
-gptq_status launch_gemm_f32(const GemmArgs& g, cudaStream_t stream);
+gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream);
+
+// x -> (tf32(x), x - tf32(x)) for a rows x cols block.
+gptq_status launch_split_tf32(const float* X, int64_t ldx, int64_t rows, int64_t cols, float* big,
+                              float* small, int64_t ldo, cudaStream_t stream);
 
 // S2-S5
 size_t prepare_workspace_bytes(int64_t cols);

@@ -8,7 +8,8 @@
 // Route: H_d = L L^T (blocked right-looking Cholesky, 128-wide panels), L^-1 (blocked triangular
 // inverse, row block by row block), H_d^-1 = L^-T L^-1 (triangular product, lower half only),
 // H_d^-1 = L2 L2^T (second Cholesky), R = L2^T. Each 128 x 128 diagonal block is factored and
-// inverted on chip by one CTA; everything else is a matrix product.
+// inverted on chip by one CTA; everything else is a 3xTF32 tensor-core matrix product whose
+// operands are kept as tf32 (big, small) pairs in the workspace.
 #include <cmath>
 
 #include "common.cuh"
@@ -20,77 +21,19 @@ namespace la {
 constexpr int kNB = 128;       // panel / diagonal block width
 constexpr int kLd = kNB + 1;   // padded shared-memory row
 constexpr int kDiagThreads = 512;
-constexpr int kDiagSmem = 2 * kNB * kLd * 4;
+constexpr int kDiagSmem = (2 * kNB * kLd + 3 * 32 * 33) * 4;
 }  // namespace la
 
-// ------------------------------------------------------------------------------------------------
-// fp32 matrix product (CUDA cores), 64 x 64 tiles, 4 x 4 outputs per thread.
-// ------------------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) gemm_f32_kernel(GemmArgs g) {
-  const int m0 = blockIdx.y * 64, n0 = blockIdx.x * 64;
-  if (g.lower && n0 > m0 + 63) return;
-  int klo = 0;
-  if (g.klo_from_m) klo = max(klo, m0);
-  if (g.klo_from_n) klo = max(klo, n0);
-  __shared__ float As[16][64 + 4];
-  __shared__ float Bs[16][64 + 4];
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
-  float acc[4][4] = {};
-  for (int k0 = klo; k0 < g.K; k0 += 16) {
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int e = tid + r * 256;
-      int mm, kk;
-      if (g.transA) { kk = e >> 6; mm = e & 63; } else { mm = e >> 4; kk = e & 15; }
-      const int m = m0 + mm, k = k0 + kk;
-      float v = 0.f;
-      if (m < g.M && k < g.K)
-        v = g.transA ? g.A[static_cast<int64_t>(k) * g.lda + m] : g.A[static_cast<int64_t>(m) * g.lda + k];
-      As[kk][mm] = v;
-      int nn;
-      if (g.transB) { nn = e >> 4; kk = e & 15; } else { kk = e >> 6; nn = e & 63; }
-      const int n = n0 + nn, k2 = k0 + kk;
-      float w = 0.f;
-      if (n < g.N && k2 < g.K)
-        w = g.transB ? g.B[static_cast<int64_t>(n) * g.ldb + k2] : g.B[static_cast<int64_t>(k2) * g.ldb + n];
-      Bs[kk][nn] = w;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int kk = 0; kk < 16; ++kk) {
-      float a[4], b[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) { a[u] = As[kk][ty * 4 + u]; b[u] = Bs[kk][tx * 4 + u]; }
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(a[u], b[v], acc[u][v]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const int m = m0 + ty * 4 + u;
-    if (m >= g.M) continue;
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int n = n0 + tx * 4 + v;
-      if (n >= g.N) continue;
-      float* c = g.C + static_cast<int64_t>(m) * g.ldc + n;
-      const float r = g.alpha * acc[u][v];
-      *c = (g.beta != 0.f) ? fmaf(g.beta, *c, r) : r;
-    }
-  }
-}
+#define GPTQ_TRY(x)               \
+  do {                            \
+    gptq_status _s = (x);         \
+    if (_s != GPTQ_OK) return _s; \
+  } while (0)
 
-gptq_status launch_gemm_f32(const GemmArgs& g, cudaStream_t stream) {
-  if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
-  dim3 grid((g.N + 63) / 64, (g.M + 63) / 64);
-  if (grid.y > 65535) return GPTQ_EUNSUPPORTED;
-  gemm_f32_kernel<<<grid, 256, 0, stream>>>(g);
-  count_launch();
-  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+__device__ __forceinline__ float tf32_rna(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -178,70 +121,225 @@ __global__ void __launch_bounds__(256) transpose_to_upper_kernel(float* R, int64
 }
 
 // ------------------------------------------------------------------------------------------------
-// S3/S5 diagonal block: Cholesky of A[k0:k0+nb, k0:k0+nb] in shared memory (lower; its strict upper
-// part is zeroed in A) and the block's triangular inverse into Dinv (ld ldd). A pivot that is not
-// positive records info_base + k0 + j + 1 and is replaced by 1 so the rest stays finite.
+// S3/S5 diagonal block: Cholesky of A[k0:k0+nb, k0:k0+nb] on chip (lower; the block's strict upper
+// part is zeroed in A) and the tf32 split of its triangular inverse into (Db, Ds) with ld ldd.
+// Blocked by 32: warp 0 factors each 32 x 32 diagonal piece with its rows in registers (the pivot
+// column is shared through shared memory, pivots use rsqrt and their reciprocals are kept), then
+// inverts the piece while warps 1-3 solve the rows below it by forward substitution; all warps
+// update the trailing part. The off-diagonal pieces of the inverse follow from
+// X[bi][bj] = -X[bi][bi] * sum_k L[bi][k] X[k][bj]. A pivot that is not positive records
+// info_base + k0 + j + 1 and is replaced by 1 so the remaining arithmetic stays finite.
 // ------------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(la::kDiagThreads)
-potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Dinv, int64_t ldd, int32_t* info,
-                  int info_base) {
-  using namespace la;
+potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, int64_t ldd,
+                  int32_t* info, int info_base) {
+  constexpr int NB = 128, LD = 129;
   extern __shared__ float sm[];
   float* L = sm;
-  float* X = sm + kNB * kLd;
+  float* X = sm + NB * LD;
+  float* T = sm + 2 * NB * LD;     // [3][32][33]
+  __shared__ float rdiag[NB];      // 1 / L[j][j]
   __shared__ int bad;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nwarps = blockDim.x >> 5;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int NW = 16;
   if (tid == 0) bad = -1;
-  for (int e = tid; e < kNB * kNB; e += blockDim.x) {
-    const int i = e / kNB, j = e % kNB;
-    float v;
-    if (i < nb && j < nb) v = (j <= i) ? A[(k0 + i) * lda + k0 + j] : 0.f;
-    else v = (i == j) ? 1.f : 0.f;
-    L[i * kLd + j] = v;
+  const bool vec = ((lda & 3) == 0) && ((k0 & 3) == 0) && ((ldd & 3) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(A) & 15) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(Db) & 15) == 0) &&
+                   ((reinterpret_cast<uintptr_t>(Ds) & 15) == 0);
+#pragma unroll 4
+  for (int e = tid; e < NB * NB / 4; e += 512) {
+    const int i = e >> 5, j = (e & 31) * 4;
+    float v[4];
+    if (vec && i < nb && j + 3 < nb) {
+      const float4 q = *reinterpret_cast<const float4*>(A + (k0 + i) * lda + k0 + j);
+      v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[u] = (i < nb && j + u < nb) ? A[(k0 + i) * lda + k0 + j + u] : (i == j + u ? 1.f : 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) L[i * LD + j + u] = (j + u <= i) ? v[u] : 0.f;
   }
   __syncthreads();
-  for (int j = 0; j < kNB; ++j) {
-    const float d = L[j * kLd + j];
-    const bool ok = d > 0.f && d < INFINITY;
-    const float ljj = ok ? sqrtf(d) : 1.f;
-    if (!ok && tid == 0 && bad < 0) bad = j;
-    const float inv = 1.f / ljj;
-    for (int i = j + 1 + tid; i < kNB; i += blockDim.x) L[i * kLd + j] *= inv;
+  for (int kb = 0; kb < 4; ++kb) {
+    const int c0 = kb * 32;
+    if (warp == 0) {
+      // lane l owns row c0 + l of the 32 x 32 piece, in registers; the pivot column goes through
+      // shared memory so each step reads it with broadcast loads
+      float d[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) d[k] = L[(c0 + lane) * LD + c0 + k];
+      float* col = T;  // 32-float scratch
+#pragma unroll 32
+      for (int j = 0; j < 32; ++j) {
+        const float piv = __shfl_sync(0xffffffffu, d[j], j);
+        const bool ok = piv > 0.f && piv < INFINITY;
+        const float r = ok ? rsqrtf(piv) : 1.f;
+        const float ljj = ok ? piv * r : 1.f;
+        if (lane == 0) {
+          if (!ok && bad < 0) bad = c0 + j;
+          rdiag[c0 + j] = r;
+        }
+        const float a = (lane == j) ? ljj : (lane > j ? d[j] * r : 0.f);
+        d[j] = a;
+        col[lane] = a;
+        __syncwarp();
+#pragma unroll 32
+        for (int k = 0; k < 32; ++k)
+          if (k > j && lane >= k) d[k] = fmaf(-a, col[k], d[k]);
+        __syncwarp();
+      }
+#pragma unroll
+      for (int k = 0; k < 32; ++k) L[(c0 + lane) * LD + c0 + k] = (k <= lane) ? d[k] : 0.f;
+    }
     __syncthreads();
-    if (tid == 0) L[j * kLd + j] = ljj;
-    for (int i = j + 1 + warp; i < kNB; i += nwarps) {
-      const float lij = L[i * kLd + j];
-      for (int l = j + 1 + lane; l <= i; l += 32) L[i * kLd + l] -= lij * L[l * kLd + j];
+    if (warp == 0) {
+      // inverse of the piece: lane t computes column t
+      float x[32];
+#pragma unroll 32
+      for (int i = 0; i < 32; ++i) {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll 32
+        for (int m = 0; m < 32; m += 2) {
+          if (m < i && m >= lane) s0 = fmaf(L[(c0 + i) * LD + c0 + m], x[m], s0);
+          if (m + 1 < i && m + 1 >= lane) s1 = fmaf(L[(c0 + i) * LD + c0 + m + 1], x[m + 1], s1);
+        }
+        x[i] = (i < lane) ? 0.f : (((i == lane) ? 1.f : 0.f) - (s0 + s1)) * rdiag[c0 + i];
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i) X[(c0 + i) * LD + c0 + lane] = x[i];
+    } else if (c0 + 32 + (warp - 1) * 32 < NB) {
+      // panel below the piece: x P^T = a by forward substitution, lane = row
+      const int r = c0 + 32 + (warp - 1) * 32 + lane;
+      float x[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) x[c] = L[r * LD + c0 + c];
+#pragma unroll 32
+      for (int c = 0; c < 32; ++c) {
+        float s0 = x[c], s1 = 0.f;
+#pragma unroll 32
+        for (int m = 0; m < 32; m += 2) {
+          if (m < c) s0 = fmaf(-x[m], L[(c0 + c) * LD + c0 + m], s0);
+          if (m + 1 < c) s1 = fmaf(-x[m + 1], L[(c0 + c) * LD + c0 + m + 1], s1);
+        }
+        x[c] = (s0 + s1) * rdiag[c0 + c];
+      }
+#pragma unroll
+      for (int c = 0; c < 32; ++c) L[r * LD + c0 + c] = x[c];
+    }
+    __syncthreads();
+    // trailing update: lane owns column l (panel values in registers); rows i >= l in steps of 4,
+    // two rows at a time
+    {
+      const int base = c0 + 32;
+      const int ncol = NB - base;
+      for (int t = warp * 32; t < ncol * 4; t += NW * 32) {
+        const int item = t + lane;
+        if (item < ncol * 4) {
+          const int l = base + item % ncol;
+          const int g = item / ncol;
+          float pv[32];
+#pragma unroll
+          for (int m = 0; m < 32; ++m) pv[m] = L[l * LD + c0 + m];
+          int i = l + g;
+          for (; i + 4 < NB; i += 8) {
+            float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 32; m += 2) {
+              s0 = fmaf(L[i * LD + c0 + m], pv[m], s0);
+              s1 = fmaf(L[i * LD + c0 + m + 1], pv[m + 1], s1);
+              u0 = fmaf(L[(i + 4) * LD + c0 + m], pv[m], u0);
+              u1 = fmaf(L[(i + 4) * LD + c0 + m + 1], pv[m + 1], u1);
+            }
+            L[i * LD + l] -= s0 + s1;
+            L[(i + 4) * LD + l] -= u0 + u1;
+          }
+          if (i < NB) {
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < 32; m += 2) {
+              s0 = fmaf(L[i * LD + c0 + m], pv[m], s0);
+              s1 = fmaf(L[i * LD + c0 + m + 1], pv[m + 1], s1);
+            }
+            L[i * LD + l] -= s0 + s1;
+          }
+        }
+      }
     }
     __syncthreads();
   }
   if (tid == 0 && bad >= 0 && bad < nb) record_info(info, info_base + k0 + bad + 1);
-  // inverse by forward substitution on all columns at once: 4 threads per column
-  {
-    const int t = tid >> 2, part = tid & 3;
-    for (int i = 0; i < kNB; ++i) {
-      float s = 0.f;
-      if (t < i)
-        for (int m = t + part; m < i; m += 4) s = fmaf(L[i * kLd + m], X[m * kLd + t], s);
-      s += __shfl_xor_sync(0xffffffffu, s, 1);
-      s += __shfl_xor_sync(0xffffffffu, s, 2);
-      if (part == 0) {
-        float x = 0.f;
-        if (t <= i) x = ((t == i ? 1.f : 0.f) - s) / L[i * kLd + i];
-        X[i * kLd + t] = x;
+  // off-diagonal pieces of the inverse, 2 x 2 outputs per thread (rows r, r+16; cols c, c+16)
+  for (int bi = 1; bi < 4; ++bi) {
+    for (int e = tid; e < bi * 256; e += 512) {
+      const int bj = e >> 8, r = (e >> 4) & 15, c = e & 15;
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+      const float* l0 = L + (32 * bi + r) * LD;
+      const float* l1 = L + (32 * bi + r + 16) * LD;
+      for (int k = 32 * bj; k < 32 * bi; ++k) {
+        const float x0 = X[k * LD + 32 * bj + c], x1 = X[k * LD + 32 * bj + c + 16];
+        const float p0 = l0[k], p1 = l1[k];
+        a00 = fmaf(p0, x0, a00); a01 = fmaf(p0, x1, a01);
+        a10 = fmaf(p1, x0, a10); a11 = fmaf(p1, x1, a11);
       }
-      __syncthreads();
+      float* t = T + bj * 32 * 33;
+      t[r * 33 + c] = a00; t[r * 33 + c + 16] = a01;
+      t[(r + 16) * 33 + c] = a10; t[(r + 16) * 33 + c + 16] = a11;
     }
+    __syncthreads();
+    for (int e = tid; e < bi * 256; e += 512) {
+      const int bj = e >> 8, r = (e >> 4) & 15, c = e & 15;
+      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
+      const float* x0r = X + (32 * bi + r) * LD + 32 * bi;
+      const float* x1r = X + (32 * bi + r + 16) * LD + 32 * bi;
+      const float* t = T + bj * 32 * 33;
+#pragma unroll 8
+      for (int m = 0; m < 32; ++m) {
+        const float t0 = t[m * 33 + c], t1 = t[m * 33 + c + 16];
+        const float p0 = x0r[m], p1 = x1r[m];
+        a00 = fmaf(p0, t0, a00); a01 = fmaf(p0, t1, a01);
+        a10 = fmaf(p1, t0, a10); a11 = fmaf(p1, t1, a11);
+      }
+      float* xo = X + (32 * bi) * LD + 32 * bj;
+      xo[r * LD + c] = -a00; xo[r * LD + c + 16] = -a01;
+      xo[(r + 16) * LD + c] = -a10; xo[(r + 16) * LD + c + 16] = -a11;
+    }
+    __syncthreads();
   }
-  for (int e = tid; e < nb * nb; e += blockDim.x) {
-    const int i = e / nb, j = e % nb;
-    A[(k0 + i) * lda + k0 + j] = (j <= i) ? L[i * kLd + j] : 0.f;
-    Dinv[i * ldd + j] = X[i * kLd + j];
+#pragma unroll 4
+  for (int e = tid; e < NB * NB / 4; e += 512) {
+    const int i = e >> 5, j = (e & 31) * 4;
+    if (i >= nb) continue;
+    float lv[4], bv[4], sv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int jj = j + u;
+      lv[u] = (jj <= i) ? L[i * LD + jj] : 0.f;
+      const float x = ((jj >> 5) <= (i >> 5)) ? X[i * LD + jj] : 0.f;
+      bv[u] = tf32_rna(x);
+      sv[u] = x - bv[u];
+    }
+    if (vec && j + 3 < nb) {
+      *reinterpret_cast<float4*>(A + (k0 + i) * lda + k0 + j) = make_float4(lv[0], lv[1], lv[2], lv[3]);
+      *reinterpret_cast<float4*>(Db + i * ldd + j) = make_float4(bv[0], bv[1], bv[2], bv[3]);
+      *reinterpret_cast<float4*>(Ds + i * ldd + j) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (j + u >= nb) continue;
+        A[(k0 + i) * lda + k0 + j + u] = lv[u];
+        Db[i * ldd + j + u] = bv[u];
+        Ds[i * ldd + j + u] = sv[u];
+      }
+    }
   }
 }
 
-static gptq_status launch_potrf_diag(float* A, int64_t n, int k0, int nb, float* Dinv, int64_t ldd,
-                                     int32_t* info, int info_base, cudaStream_t stream) {
+static gptq_status launch_potrf_diag(float* A, int64_t n, int k0, int nb, float* Db, float* Ds,
+                                     int64_t ldd, int32_t* info, int info_base,
+                                     cudaStream_t stream) {
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(potrf_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -249,101 +347,123 @@ static gptq_status launch_potrf_diag(float* A, int64_t n, int k0, int nb, float*
       return GPTQ_ECUDA;
     attr_done = true;
   }
-  potrf_diag_kernel<<<1, la::kDiagThreads, la::kDiagSmem, stream>>>(A, n, k0, nb, Dinv, ldd, info,
+  potrf_diag_kernel<<<1, la::kDiagThreads, la::kDiagSmem, stream>>>(A, n, k0, nb, Db, Ds, ldd, info,
                                                                      info_base);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }
 
-#define GPTQ_TRY(x)                       \
-  do {                                    \
-    gptq_status _s = (x);                 \
-    if (_s != GPTQ_OK) return _s;         \
-  } while (0)
+struct Split {
+  float* b;
+  float* s;
+};
 
-// Blocked right-looking Cholesky of A (n x n, lower, in place). The inverse of each diagonal block
-// of L goes to dinv_dst + k0 * (ld_dinv + 1) when per_block_dst is set (so the block diagonal of
-// L^-1 is produced for free), else to the same scratch block every panel.
-static gptq_status potrf_blocked(float* A, int64_t n, float* dinv_base, int64_t ld_dinv,
-                                 bool per_block_dst, float* panel, int32_t* info, int info_base,
+// Blocked right-looking Cholesky of A (n x n, lower, in place).
+//   Lsp:  tf32 split of L's panels (n x n, ld n), written as the panels are solved;
+//   Dsp:  where each diagonal block's inverse goes (ld ld_dinv): at block k0 of an n x n matrix
+//         when per_block is set (the block diagonal of L^-1), else one shared 128 x 128 scratch;
+//   Psp:  split of the current panel before its solve (n x 128).
+static gptq_status potrf_blocked(float* A, int64_t n, Split Lsp, Split Dsp, int64_t ld_dinv,
+                                 bool per_block, Split Psp, int32_t* info, int info_base,
                                  cudaStream_t stream) {
   using namespace la;
   for (int64_t k0 = 0; k0 < n; k0 += kNB) {
     const int nb = static_cast<int>(n - k0 < kNB ? n - k0 : kNB);
-    float* dinv = per_block_dst ? dinv_base + k0 * ld_dinv + k0 : dinv_base;
-    GPTQ_TRY(launch_potrf_diag(A, n, static_cast<int>(k0), nb, dinv, ld_dinv, info, info_base,
-                               stream));
+    const int64_t doff = per_block ? k0 * ld_dinv + k0 : 0;
+    GPTQ_TRY(launch_potrf_diag(A, n, static_cast<int>(k0), nb, Dsp.b + doff, Dsp.s + doff, ld_dinv,
+                               info, info_base, stream));
     const int64_t m = n - k0 - nb;
     if (m == 0) break;
-    // panel solve: P = A21 * L11^-T = A21 * Dinv^T
-    GemmArgs t{A + (k0 + nb) * n + k0, n, 0, dinv, ld_dinv, 1, panel, kNB,
-               static_cast<int>(m), nb, nb, 1.f, 0.f, 0, 0, 0};
-    GPTQ_TRY(launch_gemm_f32(t, stream));
-    if (cudaMemcpy2DAsync(A + (k0 + nb) * n + k0, n * sizeof(float), panel, kNB * sizeof(float),
-                          nb * sizeof(float), m, cudaMemcpyDeviceToDevice, stream) != cudaSuccess)
-      return GPTQ_ECUDA;
-    // trailing update: A22 -= P P^T (lower tiles)
-    GemmArgs u{panel, kNB, 0, panel, kNB, 1, A + (k0 + nb) * n + (k0 + nb), n,
-               static_cast<int>(m), static_cast<int>(m), nb, -1.f, 1.f, 1, 0, 0};
-    GPTQ_TRY(launch_gemm_f32(u, stream));
+    float* A21 = A + (k0 + nb) * n + k0;
+    GPTQ_TRY(launch_split_tf32(A21, n, m, nb, Psp.b, Psp.s, kNB, stream));
+    // panel solve: L21 = A21 * Dinv^T, written to A and, split, to Lsp
+    const int64_t loff = (k0 + nb) * n + k0;
+    TcGemmArgs t{Psp.b, Psp.s, Dsp.b + doff, Dsp.s + doff, kNB, ld_dinv, 0, 0,
+                 static_cast<int>(m), nb, nb, 1.f, 0.f, 0, 0, 0,
+                 A21, n, Lsp.b + loff, Lsp.s + loff, n, info};
+    GPTQ_TRY(launch_gemm_tc(t, stream));
+    // trailing update: A22 -= L21 L21^T (lower tiles)
+    TcGemmArgs u{Lsp.b + loff, Lsp.s + loff, Lsp.b + loff, Lsp.s + loff, n, n, 0, 0,
+                 static_cast<int>(m), static_cast<int>(m), nb, -1.f, 1.f, 1, 0, 0,
+                 A + (k0 + nb) * n + (k0 + nb), n, nullptr, nullptr, 0, info};
+    GPTQ_TRY(launch_gemm_tc(u, stream));
   }
   return GPTQ_OK;
 }
 
+namespace {
+struct PrepareWs {
+  Split L, V, P, T, D;
+  float* lam;
+};
+
+PrepareWs carve(void* ws, int64_t n) {
+  using namespace la;
+  uint8_t* p = static_cast<uint8_t*>(ws);
+  auto take = [&](size_t bytes) {
+    float* r = reinterpret_cast<float*>(p);
+    p += align_up(bytes, 256);
+    return r;
+  };
+  PrepareWs w;
+  const size_t nn = static_cast<size_t>(n) * n * 4, np = static_cast<size_t>(n) * kNB * 4;
+  w.L.b = take(nn); w.L.s = take(nn);
+  w.V.b = take(nn); w.V.s = take(nn);
+  w.P.b = take(np); w.P.s = take(np);
+  w.T.b = take(np); w.T.s = take(np);
+  w.D.b = take(kNB * kNB * 4); w.D.s = take(kNB * kNB * 4);
+  w.lam = take(256);
+  return w;
+}
+}  // namespace
+
 size_t prepare_workspace_bytes(int64_t cols) {
   const size_t n = static_cast<size_t>(cols);
-  size_t b = align_up(n * n * 4, 256);             // L^-1
-  b += align_up(n * la::kNB * 4, 256);             // panel / row-block scratch
-  b += align_up(la::kNB * la::kNB * 4, 256);       // diagonal-block inverse scratch
-  b += 256;                                        // lambda
-  return b;
+  return 4 * align_up(n * n * 4, 256) + 4 * align_up(n * la::kNB * 4, 256) +
+         2 * align_up(la::kNB * la::kNB * 4, 256) + 256;
 }
 
 gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, float damp_rel,
                              void* ws, int32_t* info, cudaStream_t stream) {
   using namespace la;
-  uint8_t* p = static_cast<uint8_t*>(ws);
-  float* Linv = reinterpret_cast<float*>(p);
-  p += align_up(static_cast<size_t>(n) * n * 4, 256);
-  float* panel = reinterpret_cast<float*>(p);
-  p += align_up(static_cast<size_t>(n) * kNB * 4, 256);
-  float* dscratch = reinterpret_cast<float*>(p);
-  p += align_up(kNB * kNB * 4, 256);
-  float* lam = reinterpret_cast<float*>(p);
+  PrepareWs w = carve(ws, n);
 
   // S2
   const double scale = 2.0 / static_cast<double>(n_total);
-  diag_lambda_kernel<<<1, 1024, 0, stream>>>(S_H, n, scale, damp_rel, lam, info);
+  diag_lambda_kernel<<<1, 1024, 0, stream>>>(S_H, n, scale, damp_rel, w.lam, info);
   count_launch();
   if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
   const int nt = static_cast<int>((n + 31) / 32);
   const int ntri = nt * (nt + 1) / 2;
-  finalize_kernel<<<ntri, dim3(32, 8), 0, stream>>>(S_H, R, n, static_cast<float>(scale), lam);
+  finalize_kernel<<<ntri, dim3(32, 8), 0, stream>>>(S_H, R, n, static_cast<float>(scale), w.lam);
   count_launch();
   if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
 
-  // S3: H_d = L L^T in R; diagonal blocks of L^-1 straight into Linv
-  GPTQ_TRY(potrf_blocked(R, n, Linv, n, true, panel, info, 0, stream));
+  // S3: H_d = L L^T in R; the inverses of L's diagonal blocks land in V (the split of L^-1)
+  GPTQ_TRY(potrf_blocked(R, n, w.L, w.V, n, true, w.P, info, 0, stream));
 
-  // S4a: rest of L^-1, row block by row block:
-  //   Linv[i, :i] = -Linv[i, i] * (L[i, :i] * Linv[:i, :i])
+  // S4a: the rest of L^-1, row block by row block:
+  //   T = L[i, :i] * Linv[:i, :i];  Linv[i, :i] = -Linv[i, i] * T
   for (int64_t r0 = kNB; r0 < n; r0 += kNB) {
     const int rb = static_cast<int>(n - r0 < kNB ? n - r0 : kNB);
-    GemmArgs t{R + r0 * n, n, 0, Linv, n, 0, panel, n, rb, static_cast<int>(r0),
-               static_cast<int>(r0), 1.f, 0.f, 0, 0, 1};
-    GPTQ_TRY(launch_gemm_f32(t, stream));
-    GemmArgs u{Linv + r0 * n + r0, n, 0, panel, n, 0, Linv + r0 * n, n, rb, static_cast<int>(r0),
-               rb, -1.f, 0.f, 0, 0, 0};
-    GPTQ_TRY(launch_gemm_f32(u, stream));
+    TcGemmArgs t{w.L.b + r0 * n, w.L.s + r0 * n, w.V.b, w.V.s, n, n, 0, 1,
+                 rb, static_cast<int>(r0), static_cast<int>(r0), 1.f, 0.f, 0, 0, 1,
+                 nullptr, 0, w.T.b, w.T.s, n, info};
+    GPTQ_TRY(launch_gemm_tc(t, stream));
+    TcGemmArgs u{w.V.b + r0 * n + r0, w.V.s + r0 * n + r0, w.T.b, w.T.s, n, n, 0, 1,
+                 rb, static_cast<int>(r0), rb, -1.f, 0.f, 0, 0, 0,
+                 nullptr, 0, w.V.b + r0 * n, w.V.s + r0 * n, n, info};
+    GPTQ_TRY(launch_gemm_tc(u, stream));
   }
 
   // S4b: H_d^-1 = L^-T L^-1 (lower tiles) into R
-  GemmArgs h{Linv, n, 1, Linv, n, 0, R, n, static_cast<int>(n), static_cast<int>(n),
-             static_cast<int>(n), 1.f, 0.f, 1, 1, 0};
-  GPTQ_TRY(launch_gemm_f32(h, stream));
+  TcGemmArgs h{w.V.b, w.V.s, w.V.b, w.V.s, n, n, 1, 1,
+               static_cast<int>(n), static_cast<int>(n), static_cast<int>(n), 1.f, 0.f, 1, 1, 0,
+               R, n, nullptr, nullptr, 0, info};
+  GPTQ_TRY(launch_gemm_tc(h, stream));
 
-  // S5: H_d^-1 = L2 L2^T, then R = L2^T
-  GPTQ_TRY(potrf_blocked(R, n, dscratch, kNB, false, panel, info, static_cast<int>(n), stream));
+  // S5: H_d^-1 = L2 L2^T (reusing the L split and the diagonal scratch), then R = L2^T
+  GPTQ_TRY(potrf_blocked(R, n, w.L, w.D, kNB, false, w.P, info, static_cast<int>(n), stream));
   transpose_to_upper_kernel<<<ntri, dim3(32, 8), 0, stream>>>(R, n);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;

@@ -24,6 +24,13 @@ namespace gptq {
 
 constexpr int kTPR = 8;  // lanes per weight row
 
+// tf32 rounding, for the (big, small) operand split of the trailing product
+__device__ __forceinline__ float tf32_rna_q(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
 // Grid of the asymmetric min/max quantizer (IEEE float32, each step rounded once).
 __device__ __forceinline__ void grid_params(float lo, float hi, float maxq, float& s, float& z) {
   lo = fminf(lo, 0.f);
@@ -86,7 +93,8 @@ __global__ void __launch_bounds__(128)
 column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const float* __restrict__ R,
                    int b0, int nb, int bits, int group, int group_mode, int gi_fixed,
                    float* __restrict__ scales, uint8_t* __restrict__ zeros, int G,
-                   uint8_t* __restrict__ codes, float* __restrict__ E, float* __restrict__ err_sq) {
+                   uint8_t* __restrict__ codes, float* __restrict__ Eb, float* __restrict__ Es,
+                   float* __restrict__ err_sq) {
   constexpr int CPL = B / kTPR;  // columns per lane
   extern __shared__ __align__(16) float qsm[];
   float (*Rz)[B] = reinterpret_cast<float (*)[B]>(qsm);
@@ -175,22 +183,26 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
     if (c < nb) {
       Wh[row * cols + b0 + c] = v[k];
       codes[row * cols + b0 + c] = q8[k];
-      E[row * B + c] = err[k];
+      const float eb = tf32_rna_q(err[k]);
+      Eb[row * B + c] = eb;
+      Es[row * B + c] = err[k] - eb;
     }
   }
   if (sub == 0 && err_sq != nullptr) err_sq[row] += sq;
 }
 
+// Workspace: the tf32 split of E (rows x block, twice) and of the current block's rows of R
+// (block x cols, twice).
 size_t quantize_workspace_bytes(int64_t rows, int64_t cols, int block) {
-  (void)cols;
-  return align_up(static_cast<size_t>(rows) * block * 4, 256);
+  return 2 * align_up(static_cast<size_t>(rows) * block * 4, 256) +
+         2 * align_up(static_cast<size_t>(block) * cols * 4, 256);
 }
 
 template <int B>
 static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, const float* R, int b0,
                                       int nb, int bits, int group, int group_mode, int gi_fixed,
                                       float* scales, uint8_t* zeros, int G, uint8_t* codes,
-                                      float* E, float* err_sq, cudaStream_t stream) {
+                                      float* Eb, float* Es, float* err_sq, cudaStream_t stream) {
   const int rows_per_cta = 128 / kTPR;
   const int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
   constexpr int smem = (B * B + B) * 4;
@@ -202,8 +214,8 @@ static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, con
     attr_done = true;
   }
   column_loop_kernel<B><<<static_cast<unsigned>(grid), 128, smem, stream>>>(
-      Wh, rows, cols, R, b0, nb, bits, group, group_mode, gi_fixed, scales, zeros, G, codes, E,
-      err_sq);
+      Wh, rows, cols, R, b0, nb, bits, group, group_mode, gi_fixed, scales, zeros, G, codes, Eb,
+      Es, err_sq);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }
@@ -212,8 +224,13 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
                                int64_t ldw, const float* R, int bits, int group, int block,
                                float* Wh, uint8_t* codes, float* scales, uint8_t* zeros,
                                float* err_sq, void* ws, int32_t* info, cudaStream_t stream) {
-  (void)info;
-  float* E = static_cast<float*>(ws);
+  uint8_t* wp = static_cast<uint8_t*>(ws);
+  const size_t e_bytes = align_up(static_cast<size_t>(rows) * block * 4, 256);
+  const size_t r_bytes = align_up(static_cast<size_t>(block) * cols * 4, 256);
+  float* Eb = reinterpret_cast<float*>(wp);
+  float* Es = reinterpret_cast<float*>(wp + e_bytes);
+  float* Rb = reinterpret_cast<float*>(wp + 2 * e_bytes);
+  float* Rs = reinterpret_cast<float*>(wp + 2 * e_bytes + r_bytes);
   const int G = group > 0 ? static_cast<int>(cols / group) : 1;
   const int64_t total = rows * cols;
   const int cgrid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 8 * 148));
@@ -251,24 +268,28 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
     switch (block) {
       case 32:
         st = launch_column_loop<32>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group, mode,
-                                    gi, scales, zeros, G, codes, E, err_sq, stream);
+                                    gi, scales, zeros, G, codes, Eb, Es, err_sq, stream);
         break;
       case 64:
         st = launch_column_loop<64>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group, mode,
-                                    gi, scales, zeros, G, codes, E, err_sq, stream);
+                                    gi, scales, zeros, G, codes, Eb, Es, err_sq, stream);
         break;
       default:
         st = launch_column_loop<128>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group,
-                                     mode, gi, scales, zeros, G, codes, E, err_sq, stream);
+                                     mode, gi, scales, zeros, G, codes, Eb, Es, err_sq, stream);
         break;
     }
     if (st != GPTQ_OK) return st;
     const int64_t b1 = b0 + nb;
     if (b1 < cols) {
-      // S8: W[:, b1:] -= E * R[b0:b1, b1:]
-      GemmArgs g{E, block, 0, R + b0 * cols + b1, cols, 0, Wh + b1, cols, static_cast<int>(rows),
-                 static_cast<int>(cols - b1), nb, -1.f, 1.f, 0, 0, 0};
-      st = launch_gemm_f32(g, stream);
+      // S8: W[:, b1:] -= E * R[b0:b1, b1:] on the tensor cores (3xTF32)
+      const int64_t nrest = cols - b1;
+      st = launch_split_tf32(R + b0 * cols + b1, cols, nb, nrest, Rb + b1, Rs + b1, cols, stream);
+      if (st != GPTQ_OK) return st;
+      TcGemmArgs g{Eb, Es, Rb + b1, Rs + b1, block, cols, 0, 1,
+                   static_cast<int>(rows), static_cast<int>(nrest), nb, -1.f, 1.f, 0, 0, 0,
+                   Wh + b1, cols, nullptr, nullptr, 0, info};
+      st = launch_gemm_tc(g, stream);
       if (st != GPTQ_OK) return st;
     }
   }

@@ -55,7 +55,7 @@ def _run(W, R, bits, group, block, noalloc):
 
 
 @pytest.mark.parametrize("call", [
-    (1024, 1024, 4, 128, 128),   # first call: 1024 rows x block 128 (512 KB of scratch)
+    (1024, 1024, 4, 128, 128),   # first call: 1024 x 1024 at block 128 (2 MiB of scratch)
     (300, 640, 3, -1, 64),       # second call: other shapes, per-row grid, ragged row count
 ])
 def test_noalloc_matches_workspace_entry_point(call):
@@ -72,7 +72,11 @@ def test_noalloc_matches_workspace_entry_point(call):
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     lib = _lib.load()
     fake = ctypes.c_void_p(0x10000)      # never touched: the size check comes first
-    rows = _lib.GPTQ_NOALLOC_SCRATCH_BYTES // (128 * 4) + 1
-    st = lib.gptq_quantize_layer_noalloc(fake, _lib.GPTQ_BF16, rows, 128, 128, fake, 4, -1, 128,
+    cols = 4096
+    rows = 1
+    while _lib.workspace_size(_lib.GPTQ_WS_QUANTIZE, rows, cols, 128) <= \
+            _lib.GPTQ_NOALLOC_SCRATCH_BYTES:
+        rows *= 2
+    st = lib.gptq_quantize_layer_noalloc(fake, _lib.GPTQ_BF16, rows, cols, cols, fake, 4, -1, 128,
                                          fake, fake, fake, fake, None, fake, None)
     assert st == _lib.GPTQ_EWORKSPACE
