@@ -3,15 +3,20 @@
 // "Part 2: Adaptive Rounding: Optimal Brain Quantizer (OBQ)", section "Goal": the input covariance
 // is the proxy Hessian; "Part 3: Adaptive Rounding: GPTQ", "Algorithm GPTQ": H = X X^T + lambda I.
 //
-// bf16 path: a persistent tcgen05 SYRK. Output is cut into 256 x 256 lower-triangle super-tiles;
-// each CTA owns one super-tile per round and walks the whole token range for it, so all CTAs read
-// the same token slab at about the same time (the slab is fetched from HBM once and served to the
-// others from L2). Per 32-token stage, TMA brings the 256-channel slabs of X for the tile's rows (A)
-// and columns (B) into shared memory with 128-byte swizzle; both operands are MN-major (channels
-// contiguous), which tcgen05 reads directly. One thread issues 2 x 2 MMAs of 128 x 256 x 16 into two
-// TMEM accumulators (the super-tile's upper and lower 128-row halves, 512 TMEM columns). Four
-// epilogue warps drain TMEM and add the tile into S; each super-tile belongs to one CTA, so the
-// result is deterministic and needs no atomics.
+// bf16 path: a persistent tcgen05 SYRK. Output is cut into 128 x 256 lower-triangle tiles; each
+// CTA owns one tile per round and walks the whole token range for it, so all CTAs read the same
+// token slab at about the same time (fetched from HBM once, served to the others from L2). Per
+// 32-token stage, TMA brings the 128 channels of the tile's rows (A) and the 256 channels of its
+// columns (B) into shared memory with 128-byte swizzle; both operands are MN-major (channels
+// contiguous), which tcgen05 reads directly, and a tile touching the diagonal reads A out of B's
+// slab. One thread issues two 128 x 256 x 16 MMAs per stage into a TMEM chunk accumulator.
+//
+// The tensor core adds each MMA's products into its fp32 accumulator with a rounding biased
+// toward zero, so the relative error of one TMEM sum grows with the number of MMAs folded into it
+// (about 6e-8 per MMA measured on B200). Every kChunkStages stages (2048 tokens) the chunk sum is
+// handed to eight epilogue warps, which add it into fp32 registers with IEEE adds while the MMAs
+// fill the other of two chunk buffers (2 x 256 TMEM columns); at the end of the tile the
+// registers are added into S once. Each tile belongs to one CTA: deterministic, no atomics.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -22,21 +27,29 @@ namespace gptq {
 
 namespace syrk {
 constexpr int kBK = 32;                    // tokens per stage
-constexpr int kStages = 6;
+constexpr int kStages = 8;
 constexpr int kBoxCh = 64;                 // channels per TMA box (128 bytes of bf16)
 constexpr int kBoxBytes = kBoxCh * kBK * 2;          // 4 KB
-constexpr int kSlabBytes = 4 * kBoxBytes;            // 256 channels x 32 tokens = 16 KB
-constexpr int kStageBytes = 2 * kSlabBytes;          // A slab + B slab
+constexpr int kABytes = 2 * kBoxBytes;               // 128 channels
+constexpr int kBBytes = 4 * kBoxBytes;               // 256 channels
+constexpr int kStageBytes = kABytes + kBBytes;       // 24 KB
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;
-constexpr int kThreads = 192;              // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
-constexpr uint32_t kTmemCols = 512;
-// The tensor core adds each 16-deep product into the fp32 accumulator with a rounding that is
-// biased toward zero, so the relative error of a TMEM sum grows with the number of MMAs folded
-// into it (about 6e-8 per MMA measured on B200). Every kKbPerFlush stages (2048 tokens) the
-// chunk sum is added into S with IEEE fp32 adds and the accumulator restarts.
-constexpr int kKbPerFlush = 64;
+constexpr int kThreads = 320;              // warp 0 TMA, warp 1 MMA, warps 2-9 fold/epilogue
+constexpr uint32_t kTmemCols = 512;        // two 128 x 256 fp32 chunk accumulators
+constexpr int kChunkStages = 64;           // 2048 tokens per TMEM chunk sum
 constexpr uint32_t kIdesc = make_idesc(/*bf16*/ 1, /*A MN-major*/ 1, /*B MN-major*/ 1, 128, 256);
 }  // namespace syrk
+
+// Lower tiles (I = 128-row block, J = 256-column block, 2J <= I + 1), numbered row-pair by
+// row-pair: rows 2a and 2a+1 each have a+1 tiles.
+__device__ __forceinline__ void decode_tile(int st, int& I, int& J) {
+  int a = static_cast<int>((sqrtf(4.0f * static_cast<float>(st) + 1.0f) - 1.0f) * 0.5f);
+  while ((a + 1) * (a + 2) <= st) ++a;
+  while (a * (a + 1) > st) --a;
+  const int rem = st - a * (a + 1);
+  I = 2 * a + rem / (a + 1);
+  J = rem % (a + 1);
+}
 
 __device__ __forceinline__ void decode_lower(int st, int& I, int& J) {
   int i = static_cast<int>((sqrtf(8.0f * static_cast<float>(st) + 1.0f) - 1.0f) * 0.5f);
@@ -48,7 +61,7 @@ __device__ __forceinline__ void decode_lower(int st, int& I, int& J) {
 
 __global__ void __launch_bounds__(syrk::kThreads, 1)
 hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ S, int cols,
-                     int n_kblocks, int kb_per_flush, int n_super, int32_t* info) {
+                     int n_kblocks, int n_tiles, int32_t* info) {
   using namespace syrk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -56,20 +69,23 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
 
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];
-  __shared__ __align__(8) uint64_t acc_full, acc_empty, mma_done;
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int n_chunks = (n_kblocks + kChunkStages - 1) / kChunkStages;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], 1);
     }
-    mbar_init(&acc_full, 1);
-    mbar_init(&acc_empty, 128);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 256);
+    }
     mbar_init(&mma_done, 1);
     abort_flag = 0;
     fence_mbarrier_init();
@@ -90,22 +106,22 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
       int s = 0;
       uint32_t ph = 0;
       long long issued = 0;
-      for (int st = blockIdx.x; st < n_super && !abort_flag; st += gridDim.x) {
+      for (int st = blockIdx.x; st < n_tiles && !abort_flag; st += gridDim.x) {
         int I, J;
-        decode_lower(st, I, J);
-        const bool diag = (I == J);
+        decode_tile(st, I, J);
+        const bool a_in_b = (I >> 1) == J;   // the tile's rows lie inside its column slab
         for (int kb = 0; kb < n_kblocks; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag, info)) goto producer_done;
           uint8_t* a = smem + s * kStageBytes;
-          uint8_t* b = a + kSlabBytes;
-          mbar_arrive_expect_tx(&full_bar[s], diag ? kSlabBytes : kStageBytes);
+          uint8_t* b = a + kABytes;
+          mbar_arrive_expect_tx(&full_bar[s], a_in_b ? kBBytes : kStageBytes);
 #pragma unroll
           for (int q = 0; q < 4; ++q)
-            tma_load_2d(a + q * kBoxBytes, &tmap, &full_bar[s], I * 256 + q * kBoxCh, kb * kBK);
-          if (!diag) {
+            tma_load_2d(b + q * kBoxBytes, &tmap, &full_bar[s], J * 256 + q * kBoxCh, kb * kBK);
+          if (!a_in_b) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              tma_load_2d(b + q * kBoxBytes, &tmap, &full_bar[s], J * 256 + q * kBoxCh, kb * kBK);
+            for (int q = 0; q < 2; ++q)
+              tma_load_2d(a + q * kBoxBytes, &tmap, &full_bar[s], I * 128 + q * kBoxCh, kb * kBK);
           }
           ++issued;
           if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -120,36 +136,34 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
       int s = 0;
-      uint32_t ph = 0, aph = 0;
-      for (int st = blockIdx.x; st < n_super && !abort_flag; st += gridDim.x) {
+      uint32_t ph = 0;
+      int chunk = 0;   // running chunk count: buffer = chunk & 1, its use = chunk >> 1
+      for (int st = blockIdx.x; st < n_tiles && !abort_flag; st += gridDim.x) {
         int I, J;
-        decode_lower(st, I, J);
-        const bool diag = (I == J);
-        for (int kc = 0; kc < n_kblocks; kc += kb_per_flush) {
-          // a fresh chunk sum in TMEM; the epilogue folds it into S with IEEE fp32 adds
-          if (!mbar_wait_bounded(&acc_empty, aph ^ 1u, &abort_flag, info)) goto mma_done_label;
+        decode_tile(st, I, J);
+        const bool a_in_b = (I >> 1) == J;
+        for (int kc = 0; kc < n_kblocks; kc += kChunkStages, ++chunk) {
+          const int buf = chunk & 1;
+          if (!mbar_wait_bounded(&acc_empty[buf], ((chunk >> 1) & 1) ^ 1u, &abort_flag, info))
+            goto mma_done_label;
           tc_fence_after();
-          const int kc_end = min(n_kblocks, kc + kb_per_flush);
+          const int kc_end = min(n_kblocks, kc + kChunkStages);
           for (int kb = kc; kb < kc_end; ++kb) {
             if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag, info)) goto mma_done_label;
             tc_fence_after();
-            const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
-            const uint32_t b_addr = diag ? a_addr : a_addr + kSlabBytes;
+            const uint32_t st_addr = smem_u32(smem + s * kStageBytes);
+            const uint32_t b_addr = st_addr + kABytes;
+            const uint32_t a_addr = a_in_b ? b_addr + (I & 1) * 2 * kBoxBytes : st_addr;
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t adesc = smem_desc(a_addr + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
               const uint64_t bdesc = smem_desc(b_addr + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const uint64_t adesc = smem_desc(a_addr + 2 * h * kBoxBytes + kk * 2048, kBoxBytes,
-                                                 1024, kSwizzle128B);
-                tc_mma_f16(tmem + h * 256, adesc, bdesc, kIdesc, (kb > kc || kk > 0) ? 1u : 0u);
-              }
+              tc_mma_f16(tmem + buf * 256, adesc, bdesc, kIdesc, (kb > kc || kk > 0) ? 1u : 0u);
             }
             tc_commit(&empty_bar[s]);
             if (++s == kStages) { s = 0; ph ^= 1u; }
           }
-          tc_commit(&acc_full);
-          aph ^= 1u;
+          tc_commit(&acc_full[buf]);
         }
       }
     mma_done_label:
@@ -157,47 +171,54 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
       mbar_drain_bounded(&mma_done, 0);
     }
   } else {
-    // ---------------- epilogue: TMEM -> S (read-add-write, lower super-tile) ----------------
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int r_in_half = q * 32 + lane;
-    uint32_t aph = 0;
-    for (int st = blockIdx.x; st < n_super && !abort_flag; st += gridDim.x) {
+    // ---------------- fold chunk sums into registers; add the tile into S at its end ----------
+    const int q = warp & 3;            // TMEM lane quarter this warp may access
+    const int h = (warp - 2) >> 2;     // column half: 0 -> 0..127, 1 -> 128..255
+    int chunk = 0;
+    bool ok = true;
+    for (int st = blockIdx.x; st < n_tiles && ok && !abort_flag; st += gridDim.x) {
       int I, J;
-      decode_lower(st, I, J);
-      for (int kc = 0; kc < n_kblocks; kc += kb_per_flush) {
-        if (!mbar_wait_bounded(&acc_full, aph, &abort_flag, info)) goto epilogue_done;
-        tc_fence_after();
-#pragma unroll 1
-        for (int h = 0; h < 2; ++h) {
-          const int i = I * 256 + h * 128 + r_in_half;
-#pragma unroll 1
-          for (int c = 0; c < 8; ++c) {
-            uint32_t v[32];
-            tmem_ld_32x32b_x32(tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 256 + c * 32, v);
-            tmem_wait_ld();
-            const int j0 = J * 256 + c * 32;
-            if (i < cols) {
-              float4* row = reinterpret_cast<float4*>(S + static_cast<size_t>(i) * cols + j0);
+      decode_tile(st, I, J);
+      float acc[128];
 #pragma unroll
-              for (int t = 0; t < 8; ++t) {
-                if (j0 + 4 * t < cols) {
-                  float4 o = row[t];
-                  o.x += __uint_as_float(v[4 * t + 0]);
-                  o.y += __uint_as_float(v[4 * t + 1]);
-                  o.z += __uint_as_float(v[4 * t + 2]);
-                  o.w += __uint_as_float(v[4 * t + 3]);
-                  row[t] = o;
-                }
-              }
-            }
-          }
+      for (int j = 0; j < 128; ++j) acc[j] = 0.f;
+      for (int kc = 0; kc < n_kblocks; kc += kChunkStages, ++chunk) {
+        const int buf = chunk & 1;
+        if (!mbar_wait_bounded(&acc_full[buf], (chunk >> 1) & 1, &abort_flag, info)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t t0 = tmem + buf * 256 + h * 128 + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(t0 + cc * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int t = 0; t < 32; ++t) acc[cc * 32 + t] += __uint_as_float(v[t]);
         }
         tc_fence_before();
-        mbar_arrive(&acc_empty);
-        aph ^= 1u;
+        mbar_arrive(&acc_empty[buf]);
+      }
+      if (!ok) break;
+      const int i = I * 128 + q * 32 + lane;
+      const int j0 = J * 256 + h * 128;
+      if (i < cols) {
+        float4* row = reinterpret_cast<float4*>(S + static_cast<size_t>(i) * cols + j0);
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          if (j0 + 4 * t < cols) {
+            float4 o = row[t];
+            o.x += acc[4 * t + 0];
+            o.y += acc[4 * t + 1];
+            o.z += acc[4 * t + 2];
+            o.w += acc[4 * t + 3];
+            row[t] = o;
+          }
+        }
       }
     }
-  epilogue_done:;
   }
 
   tc_fence_before();
@@ -278,13 +299,15 @@ gptq_status launch_hessian_bf16(float* S, int64_t cols, const void* X, int64_t n
       return GPTQ_ECUDA;
     attr_done = true;
   }
-  const int n_s = static_cast<int>((cols + 255) / 256);
-  const int n_super = n_s * (n_s + 1) / 2;
+  // lower 128 x 256 tiles: row block I has floor(I / 2) + 1 of them
+  const int n_i = static_cast<int>((cols + 127) / 128);
+  int n_tiles = 0;
+  for (int I = 0; I < n_i; ++I) n_tiles += I / 2 + 1;
   const int64_t n_kb = (n_tokens + kBK - 1) / kBK;
   if (n_kb > INT32_MAX / kBK) return GPTQ_EUNSUPPORTED;
-  const int grid = n_super < num_sms() ? n_super : num_sms();
+  const int grid = n_tiles < num_sms() ? n_tiles : num_sms();
   hessian_syrk_bf16_tc<<<grid, kThreads, kSmemBytes, stream>>>(
-      tmap, S, static_cast<int>(cols), static_cast<int>(n_kb), kKbPerFlush, n_super, info);
+      tmap, S, static_cast<int>(cols), static_cast<int>(n_kb), n_tiles, info);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }
