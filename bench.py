@@ -36,6 +36,11 @@ sys.path.insert(0, ROOT)
 METRIC = "GPTQ layer quantize: weights/sec & ms per layer (4-bit g128); % of roofline"
 UNIT = "weights/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Nominal dense tf32 / bf16 throughput ratio (1.1 / 2.25 PFLOP/s); tf32 has no measured peak here.
+TF32_PER_BF16 = 1.1 / 2.25
+# DRAM traffic of the S1 kernel from one ncu capture of 16384 tokens x 4096 channels (reads scale
+# with tokens -- X is streamed once per round of tiles; writes are S, once per launch).
+SYRK_CAPTURE = {"tokens": 16384, "cols": 4096, "dram_read": 269.261e6, "dram_write": 26.181e6}
 
 
 def parse():
@@ -229,6 +234,24 @@ def run_reference(args):
 # our arm
 # ------------------------------------------------------------------------------------------------
 
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank quantizes its own independent layer: seeds 1000 apart."""
+    return seed + 1000 * rank
+
+
+def aggregate(elapsed_ms: float, launches: int, world: int, device):
+    """Job time = max over ranks (every rank's work must finish); kernel launches = sum."""
+    if world <= 1:
+        return elapsed_ms, launches
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([elapsed_ms], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    c = torch.tensor([launches], device=device, dtype=torch.int64)
+    dist.all_reduce(c, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(c.item())
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -244,7 +267,7 @@ def run_ours(args):
                                 device_id=dev)
     peaks, peaks_src = load_peaks()
     spec = workload(args.tokens)
-    seed = args.seed + 1000 * rank
+    seed = rank_seed(args.seed, rank)
     rows, cols, n = spec.rows, spec.cols, spec.n_tokens
 
     X = synth.inputs_torch(spec, seed, dev)
@@ -312,13 +335,7 @@ def run_ours(args):
     if int(info.item()) != 0:
         raise RuntimeError(f"device status {int(info.item())} in the timed region")
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-        c = torch.tensor([launches], device=dev, dtype=torch.int64)
-        dist.all_reduce(c, op=dist.ReduceOp.SUM)
-        launches = int(c.item())
+    elapsed_ms, launches = aggregate(elapsed_ms, launches, world, dev)
 
     ms_per_step = elapsed_ms / args.steps
     value = world * rows * cols * args.steps / (elapsed_ms / 1e3)
@@ -328,11 +345,40 @@ def run_ours(args):
     flops = cols * (cols + 1) * n            # symmetric half of X^T X, 2 flops per multiply-add
     achieved = flops / t_syrk / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    traffic = None
+    if cols == SYRK_CAPTURE["cols"]:
+        traffic = SYRK_CAPTURE["dram_read"] * n / SYRK_CAPTURE["tokens"] + SYRK_CAPTURE["dram_write"]
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": traffic,
                 "kernel": "hessian_syrk_bf16_tc",
                 "peak_source": f"{peaks_src} bf16 sustained (kernel timed inside a long step)",
-                "work": f"{flops:.4g} flop per launch = cols*(cols+1)*n_tokens"}
+                "work": f"{flops:.4g} flop per launch = cols*(cols+1)*n_tokens",
+                "traffic_source": "ncu dram bytes at 16384 tokens, reads scaled by tokens"}
+
+    # Per-stage and whole-layer rooflines from the algorithmic work of each stage:
+    #   S1: cols*(cols+1)*tokens flop at the bf16 tensor peak;
+    #   S2-S5: 4/3 cols^3 fp32 flop (two Cholesky, one triangular inverse, one triangular
+    #          product), each done as 3 tf32 products: peak = tf32 peak / 3;
+    #   S6-S8: HBM bytes, 9 B per weight for the column loop (read + write fp32, code byte) plus
+    #          8 B per trailing element per block for the lazy update (fp32 read + write).
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])) * 1e9
+    tf32x3 = peak * 1e12 * TF32_PER_BF16 / 3.0
+    fl_25 = 4.0 / 3.0 * cols ** 3
+    b_trail = sum(8.0 * rows * (cols - min(cols, b0 + spec.block))
+                  for b0 in range(0, cols, spec.block))
+    b_68 = 9.0 * rows * cols + b_trail
+    ideal = {"S1_hessian": flops / (peak * 1e12), "S2_S5_factor": fl_25 / tf32x3,
+             "S6_S8_quantize": b_68 / hbm}
+    got = {"S1_hessian": statistics.mean(s1) / 1e3, "S2_S5_factor": statistics.mean(s25) / 1e3,
+           "S6_S8_quantize": statistics.mean(s68) / 1e3}
+    stage_roofline = {k: {"ideal_ms": ideal[k] * 1e3, "ms": got[k] * 1e3,
+                          "frac": ideal[k] / got[k]} for k in ideal}
+    stage_roofline["S2_S5_factor"]["achieved_tflops_fp32_equiv"] = fl_25 / got["S2_S5_factor"] / 1e12
+    stage_roofline["S6_S8_quantize"]["achieved_gbs"] = b_68 / got["S6_S8_quantize"] / 1e9
+    layer_roofline = {"ideal_ms": sum(ideal.values()) * 1e3, "ms": ms_per_step,
+                      "frac": sum(ideal.values()) * 1e3 / ms_per_step,
+                      "basis": f"{peaks_src} peaks: bf16 sustained {peak} TFLOP/s, tf32 = bf16 x "
+                               f"{TF32_PER_BF16:.3f} (nominal ratio), HBM {hbm / 1e9:.0f} GB/s"}
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -342,7 +388,8 @@ def run_ours(args):
         "config": config_dict(spec),
         "stages_ms": {"S1_hessian": statistics.mean(s1), "S2_S5_factor": statistics.mean(s25),
                       "S6_S8_quantize": statistics.mean(s68)},
-        "roofline": roofline, "gpu_launches": launches, "clocks": clock_rec,
+        "roofline": roofline, "stage_roofline": stage_roofline, "layer_roofline": layer_roofline,
+        "gpu_launches": launches, "clocks": clock_rec,
     }
     if args.tokens:
         line["note"] = "token count overridden for profiling: not the configured workload"
@@ -372,11 +419,7 @@ def run_ours(args):
             out = e2e_step()
         b.record(stream)
         torch.cuda.synchronize(dev)
-        e_ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms, _ = aggregate(a.elapsed_time(b), 0, world, dev)
         h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
         d2h = sum(t.numel() * t.element_size() for t in (out.codes, out.scales, out.zeros,
                                                          out.W_hat, out.err_sq))
