@@ -40,6 +40,17 @@ __device__ __forceinline__ void grid_params(float lo, float hi, float maxq, floa
   z = fminf(fmaxf(rintf(__fdiv_rn(-lo, s)), 0.f), maxq);
 }
 
+// rint(w / s) with the quotient rounded once in IEEE float32, as the quantizer defines it, without a
+// division in the common case: y = w * (1/s) is within ~2^-23 relative of the true quotient, so
+// when y is farther than 1e-5 |y| from a half-integer, rint(y) equals rint(fl(w / s)); otherwise
+// (rare) the correctly rounded division decides.
+__device__ __forceinline__ float rint_quot(float w, float s, float inv_s) {
+  const float y = w * inv_s;
+  const float r = rintf(y);
+  if (0.5f - fabsf(y - r) > 1e-5f * fmaxf(1.f, fabsf(y))) return r;
+  return rintf(__fdiv_rn(w, s));
+}
+
 template <typename T>
 __device__ __forceinline__ float load_w(const T* p);
 template <>
@@ -88,6 +99,10 @@ __global__ void params_kernel(const float* __restrict__ Wh, int64_t rows, int64_
 // One block of B columns [b0, b0 + nb) for every row.
 //   group_mode: 0 = grid given per row (scales[row*G + gi_fixed]);
 //               1 = groups of `group` columns inside the block, grids computed here.
+// Lane `sub` of a row holds, in registers, the columns 32*t + 4*sub + u (t < B/32, u < 4): the 8
+// lanes of a row together cover each 32-column stretch with one float4 each, so their reads of a
+// row of R and their loads/stores of W, E and codes are contiguous 128-byte segments (no shared
+// memory bank conflicts, coalesced global accesses).
 template <int B>
 __global__ void __launch_bounds__(128)
 column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const float* __restrict__ R,
@@ -95,13 +110,45 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
                    float* __restrict__ scales, uint8_t* __restrict__ zeros, int G,
                    uint8_t* __restrict__ codes, float* __restrict__ Eb, float* __restrict__ Es,
                    float* __restrict__ err_sq) {
-  constexpr int CPL = B / kTPR;  // columns per lane
+  constexpr int NT = B / 32;       // float4 groups per lane
+  constexpr int CPL = 4 * NT;      // columns per lane
   extern __shared__ __align__(16) float qsm[];
   float (*Rz)[B] = reinterpret_cast<float (*)[B]>(qsm);
   float* inv_d = qsm + B * B;
-  for (int e = threadIdx.x; e < B * B; e += blockDim.x) {
-    const int i = e / B, j = e % B;
-    Rz[i][j] = (i < nb && j < nb && j > i) ? R[(b0 + i) * cols + b0 + j] : 0.f;
+  // the block's corner of R with its diagonal and lower part zeroed; every load in flight at once
+  // (rows are 16-byte aligned: cols % 4 == 0, b0 % 4 == 0)
+  {
+    constexpr int PER = B * B / 4 / 128;  // float4 per thread
+    float4 buf[PER];
+#pragma unroll
+    for (int p = 0; p < PER; ++p) {
+      const int e = threadIdx.x + p * 128;
+      const int i = (4 * e) / B, j = (4 * e) % B;
+      float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < nb) {
+        const float* src = R + (b0 + i) * cols + b0 + j;
+        if (j + 3 < nb) {
+          q = *reinterpret_cast<const float4*>(src);
+        } else {
+          q.x = (j + 0 < nb) ? src[0] : 0.f;
+          q.y = (j + 1 < nb) ? src[1] : 0.f;
+          q.z = (j + 2 < nb) ? src[2] : 0.f;
+          q.w = (j + 3 < nb) ? src[3] : 0.f;
+        }
+      }
+      buf[p] = q;
+    }
+#pragma unroll
+    for (int p = 0; p < PER; ++p) {
+      const int e = threadIdx.x + p * 128;
+      const int i = (4 * e) / B, j = (4 * e) % B;
+      float4 q = buf[p];
+      q.x = (j + 0 > i) ? q.x : 0.f;
+      q.y = (j + 1 > i) ? q.y : 0.f;
+      q.z = (j + 2 > i) ? q.z : 0.f;
+      q.w = (j + 3 > i) ? q.w : 0.f;
+      *reinterpret_cast<float4*>(&Rz[i][j]) = q;
+    }
   }
   for (int i = threadIdx.x; i < B; i += blockDim.x)
     inv_d[i] = (i < nb) ? 1.f / R[(b0 + i) * cols + b0 + i] : 0.f;
@@ -112,15 +159,30 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   const int base_lane = lane & ~(kTPR - 1);
   const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x / kTPR) + threadIdx.x / kTPR;
   const bool valid = row < rows;
-  const int c_first = sub * CPL;              // first block column this lane holds
+  auto colof = [&](int k) { return 32 * (k >> 2) + 4 * sub + (k & 3); };  // block column of v[k]
 
   float v[CPL];
   uint8_t q8[CPL];
   float err[CPL];
 #pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    const int c = 32 * t + 4 * sub;
+    float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (valid) {
+      const float* src = Wh + row * cols + b0 + c;
+      if (c + 3 < nb) {
+        w4 = *reinterpret_cast<const float4*>(src);
+      } else {
+        w4.x = (c + 0 < nb) ? src[0] : 0.f;
+        w4.y = (c + 1 < nb) ? src[1] : 0.f;
+        w4.z = (c + 2 < nb) ? src[2] : 0.f;
+        w4.w = (c + 3 < nb) ? src[3] : 0.f;
+      }
+    }
+    v[4 * t + 0] = w4.x; v[4 * t + 1] = w4.y; v[4 * t + 2] = w4.z; v[4 * t + 3] = w4.w;
+  }
+#pragma unroll
   for (int k = 0; k < CPL; ++k) {
-    const int c = c_first + k;
-    v[k] = (valid && c < nb) ? Wh[row * cols + b0 + c] : 0.f;
     q8[k] = 0;
     err[k] = 0.f;
   }
@@ -130,43 +192,53 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
     s = scales[row * G + gi_fixed];
     z = static_cast<float>(zeros[row * G + gi_fixed]);
   }
+  float inv_s = 1.f / s;
 
-  for (int o = 0; o < kTPR; ++o) {
 #pragma unroll
-    for (int kk = 0; kk < CPL; ++kk) {
-      const int j = o * CPL + kk;
-      if (j < nb) {
-        if (group_mode == 1 && (j % group) == 0) {
-          float lo = 0.f, hi = 0.f;
+  for (int t = 0; t < NT; ++t) {
+    for (int o = 0; o < kTPR; ++o) {        // owner lane of columns 32t + 4o .. 32t + 4o + 3
 #pragma unroll
-          for (int k = 0; k < CPL; ++k) {
-            const int c = c_first + k;
-            if (c >= j && c < j + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
+      for (int u = 0; u < 4; ++u) {
+        const int j = 32 * t + 4 * o + u;
+        const int kk = 4 * t + u;           // register slot of column j in its owner lane
+        if (j < nb) {
+          if (group_mode == 1 && (j % group) == 0) {
+            float lo = 0.f, hi = 0.f;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+              const int c = colof(k);
+              if (c >= j && c < j + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
+            }
+#pragma unroll
+            for (int off = kTPR / 2; off > 0; off >>= 1) {
+              lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+              hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+            }
+            grid_params(lo, hi, maxq, s, z);
+            inv_s = 1.f / s;
+            if (valid && sub == 0) {
+              const int gi = (b0 + j) / group;
+              scales[row * G + gi] = s;
+              zeros[row * G + gi] = static_cast<uint8_t>(z);
+            }
           }
+          const float w = __shfl_sync(0xffffffffu, v[kk], base_lane + o);
+          const float q = fminf(fmaxf(rint_quot(w, s, inv_s) + z, 0.f), maxq);
+          const float wh = __fmul_rn(s, q - z);
+          const float e = __fmul_rn(__fsub_rn(w, wh), inv_d[j]);
+          const bool own = (sub == o);
+          v[kk] = own ? wh : v[kk];
+          q8[kk] = own ? static_cast<uint8_t>(q) : q8[kk];
+          err[kk] = own ? e : err[kk];
 #pragma unroll
-          for (int off = kTPR / 2; off > 0; off >>= 1) {
-            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-          }
-          grid_params(lo, hi, maxq, s, z);
-          if (valid && sub == 0) {
-            const int gi = (b0 + j) / group;
-            scales[row * G + gi] = s;
-            zeros[row * G + gi] = static_cast<uint8_t>(z);
+          for (int t2 = 0; t2 < NT; ++t2) {
+            const float4 r4 = *reinterpret_cast<const float4*>(&Rz[j][32 * t2 + 4 * sub]);
+            v[4 * t2 + 0] = fmaf(-e, r4.x, v[4 * t2 + 0]);
+            v[4 * t2 + 1] = fmaf(-e, r4.y, v[4 * t2 + 1]);
+            v[4 * t2 + 2] = fmaf(-e, r4.z, v[4 * t2 + 2]);
+            v[4 * t2 + 3] = fmaf(-e, r4.w, v[4 * t2 + 3]);
           }
         }
-        const float w = __shfl_sync(0xffffffffu, v[kk], base_lane + o);
-        const float q = fminf(fmaxf(rintf(__fdiv_rn(w, s)) + z, 0.f), maxq);
-        const float wh = __fmul_rn(s, q - z);
-        const float e = __fmul_rn(__fsub_rn(w, wh), inv_d[j]);
-        if (sub == o) {
-          v[kk] = wh;
-          q8[kk] = static_cast<uint8_t>(q);
-          err[kk] = e;
-        }
-        const float* rrow = &Rz[j][c_first];
-#pragma unroll
-        for (int k = 0; k < CPL; ++k) v[k] = fmaf(-e, rrow[k], v[k]);
       }
     }
   }
@@ -178,14 +250,35 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   for (int off = kTPR / 2; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
   if (!valid) return;
 #pragma unroll
-  for (int k = 0; k < CPL; ++k) {
-    const int c = c_first + k;
-    if (c < nb) {
-      Wh[row * cols + b0 + c] = v[k];
-      codes[row * cols + b0 + c] = q8[k];
-      const float eb = tf32_rna_q(err[k]);
-      Eb[row * B + c] = eb;
-      Es[row * B + c] = err[k] - eb;
+  for (int t = 0; t < NT; ++t) {
+    const int c = 32 * t + 4 * sub;
+    float* wd = Wh + row * cols + b0 + c;
+    uint8_t* cd = codes + row * cols + b0 + c;
+    float* eb = Eb + row * B + c;
+    float* es = Es + row * B + c;
+    float b4[4], s4[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      b4[u] = tf32_rna_q(err[4 * t + u]);
+      s4[u] = err[4 * t + u] - b4[u];
+    }
+    if (c + 3 < nb) {
+      *reinterpret_cast<float4*>(wd) = make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
+      *reinterpret_cast<float4*>(eb) = make_float4(b4[0], b4[1], b4[2], b4[3]);
+      *reinterpret_cast<float4*>(es) = make_float4(s4[0], s4[1], s4[2], s4[3]);
+      *reinterpret_cast<uint32_t*>(cd) =
+          static_cast<uint32_t>(q8[4 * t]) | (static_cast<uint32_t>(q8[4 * t + 1]) << 8) |
+          (static_cast<uint32_t>(q8[4 * t + 2]) << 16) | (static_cast<uint32_t>(q8[4 * t + 3]) << 24);
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (c + u < nb) {
+          wd[u] = v[4 * t + u];
+          cd[u] = q8[4 * t + u];
+          eb[u] = b4[u];
+          es[u] = s4[u];
+        }
+      }
     }
   }
   if (sub == 0 && err_sq != nullptr) err_sq[row] += sq;
