@@ -53,7 +53,22 @@ struct TcGemmParams {
   int64_t ld_split;
   int tiles_n;
   int vec4;                // C / split rows are 16-byte aligned
+  int tiles_m, n_tiles;    // used by the persistent K <= 128 variant
 };
+
+// tile index -> (tm, tn): row-major over all tiles, or over the lower triangle tn <= tm
+__device__ __forceinline__ void tile_coords(const TcGemmParams& p, int t, int& tm, int& tn) {
+  if (p.lower) {
+    int i = static_cast<int>((sqrtf(8.0f * static_cast<float>(t) + 1.0f) - 1.0f) * 0.5f);
+    while ((i + 1) * (i + 2) / 2 <= t) ++i;
+    while (i * (i + 1) / 2 > t) --i;
+    tm = i;
+    tn = t - i * (i + 1) / 2;
+  } else {
+    tm = t / p.tiles_n;
+    tn = t - tm * p.tiles_n;
+  }
+}
 
 __global__ void __launch_bounds__(tg::kThreads, 1)
 gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ CUtensorMap tAs,
@@ -260,6 +275,220 @@ gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ 
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// K <= 128 products (the lazy trailing update, the Cholesky panel solve and trailing update, the
+// triangular inverse's second product): persistent over a contiguous range of output tiles, A and
+// B streamed through two 64 KB stages. Keeping shared memory at 128 KB leaves the rest of the
+// SM's unified L1 to the epilogue, whose row-wise float4 read-modify-write of C (64 KB per tile)
+// then stays in L1; two TMEM buffers let one tile's epilogue overlap the next tile's MMAs.
+// ------------------------------------------------------------------------------------------------
+namespace tgp {
+constexpr int BM = 128, BN = 128, BK = 32;
+constexpr int kMaxK = 128;
+constexpr int kPartBytes = BM * BK * 4;             // 16 KB: one part (big or small) of one operand
+constexpr int kStages = 2;
+constexpr int kStageBytes = 4 * kPartBytes;         // A_big, A_small, B_big, B_small
+constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+}  // namespace tgp
+
+__global__ void __launch_bounds__(tgp::kThreads, 1)
+gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ CUtensorMap tAs,
+                     const __grid_constant__ CUtensorMap tBb, const __grid_constant__ CUtensorMap tBs,
+                     TcGemmParams p, int32_t* info) {
+  using namespace tgp;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = (p.K + BK - 1) / BK;   // 1..4
+  const int t_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * p.n_tiles / gridDim.x);
+  const int t_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * p.n_tiles / gridDim.x);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0;
+      int issued = 0;
+      for (int t = t_begin; t < t_end && !abort_flag; ++t) {
+        int tm, tn;
+        tile_coords(p, t, tm, tn);
+        const int m0 = tm * BM, n0 = tn * BN;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag, info)) goto producer_done;
+          uint8_t* st = smem + s * kStageBytes;
+          const int k0 = kb * BK;
+          mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
+          if (p.a_mn) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              tma_load_2d(st + q * 4096, &tAb, &full_bar[s], m0 + 32 * q, k0);
+              tma_load_2d(st + kPartBytes + q * 4096, &tAs, &full_bar[s], m0 + 32 * q, k0);
+            }
+          } else {
+            tma_load_2d(st, &tAb, &full_bar[s], k0, m0);
+            tma_load_2d(st + kPartBytes, &tAs, &full_bar[s], k0, m0);
+          }
+          if (p.b_mn) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              tma_load_2d(st + 2 * kPartBytes + q * 4096, &tBb, &full_bar[s], n0 + 32 * q, k0);
+              tma_load_2d(st + 3 * kPartBytes + q * 4096, &tBs, &full_bar[s], n0 + 32 * q, k0);
+            }
+          } else {
+            tma_load_2d(st + 2 * kPartBytes, &tBb, &full_bar[s], k0, n0);
+            tma_load_2d(st + 3 * kPartBytes, &tBs, &full_bar[s], k0, n0);
+          }
+          ++issued;
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+      }
+    producer_done:
+      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+        mbar_drain_bounded(&full_bar[i % kStages], static_cast<uint32_t>((i / kStages) & 1));
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(/*tf32*/ 2, p.a_mn, p.b_mn, BM, BN);
+      const uint32_t a_lbo = p.a_mn ? 4096u : 16u, b_lbo = p.b_mn ? 4096u : 16u;
+      const uint32_t a_sbo = p.a_mn ? 512u : 1024u, b_sbo = p.b_mn ? 512u : 1024u;
+      const uint32_t a_lay = p.a_mn ? kSwizzle128B32BAtom : kSwizzle128B;
+      const uint32_t b_lay = p.b_mn ? kSwizzle128B32BAtom : kSwizzle128B;
+      const uint32_t a_step = p.a_mn ? 1024u : 32u, b_step = p.b_mn ? 1024u : 32u;
+      int s = 0, c = 0;
+      uint32_t ph = 0;
+      for (int t = t_begin; t < t_end && !abort_flag; ++t, ++c) {
+        const int buf = c & 1;
+        if (!mbar_wait_bounded(&acc_empty[buf], ((c >> 1) & 1) ^ 1u, &abort_flag, info))
+          goto mma_done_label;
+        tc_fence_after();
+        const uint32_t t_main = tmem + buf * 256, t_corr = t_main + 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag, info)) goto mma_done_label;
+          tc_fence_after();
+          const uint32_t base = smem_u32(smem + s * kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 8; ++kk) {
+            const uint64_t ab = smem_desc(base + kk * a_step, a_lbo, a_sbo, a_lay);
+            const uint64_t as = smem_desc(base + kPartBytes + kk * a_step, a_lbo, a_sbo, a_lay);
+            const uint64_t bb = smem_desc(base + 2 * kPartBytes + kk * b_step, b_lbo, b_sbo, b_lay);
+            const uint64_t bs = smem_desc(base + 3 * kPartBytes + kk * b_step, b_lbo, b_sbo, b_lay);
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            tc_mma_tf32(t_corr, ab, bs, idesc, accum);
+            tc_mma_tf32(t_corr, as, bb, idesc, 1u);
+            tc_mma_tf32(t_main, ab, bb, idesc, accum);
+          }
+          tc_commit(&empty_bar[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+        tc_commit(&acc_full[buf]);
+      }
+    mma_done_label:
+      tc_commit(&mma_done);
+      mbar_drain_bounded(&mma_done, 0);
+    }
+  } else {
+    const int q = warp & 3;
+    int c = 0;
+    for (int t = t_begin; t < t_end && !abort_flag; ++t, ++c) {
+      int tm, tn;
+      tile_coords(p, t, tm, tn);
+      const int m0 = tm * BM, n0 = tn * BN;
+      const int buf = c & 1;
+      if (!mbar_wait_bounded(&acc_full[buf], (c >> 1) & 1, &abort_flag, info)) break;
+      tc_fence_after();
+      float acc[BN];
+      const uint32_t t_main = tmem + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t vm[32], vc[32];
+        tmem_ld_32x32b_x32(t_main + cc * 32, vm);
+        tmem_ld_32x32b_x32(t_main + 128 + cc * 32, vc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) acc[cc * 32 + u] = __uint_as_float(vm[u]) + __uint_as_float(vc[u]);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);   // the buffer is free as soon as the sums are in registers
+      const int row = m0 + q * 32 + lane;
+      if (row < p.M) {
+        float* crow = p.C ? p.C + static_cast<int64_t>(row) * p.ldc + n0 : nullptr;
+        float* brow = p.Cbig ? p.Cbig + static_cast<int64_t>(row) * p.ld_split + n0 : nullptr;
+        float* srow = p.Cbig ? p.Csmall + static_cast<int64_t>(row) * p.ld_split + n0 : nullptr;
+        const int ncol = min(BN, p.N - n0);
+        if (p.vec4 && ncol == BN) {
+#pragma unroll
+          for (int j = 0; j < BN; j += 4) {
+            float4 v = make_float4(p.alpha * acc[j], p.alpha * acc[j + 1], p.alpha * acc[j + 2],
+                                   p.alpha * acc[j + 3]);
+            if (p.beta != 0.f) {
+              const float4 o = *reinterpret_cast<const float4*>(crow + j);
+              v.x = fmaf(p.beta, o.x, v.x); v.y = fmaf(p.beta, o.y, v.y);
+              v.z = fmaf(p.beta, o.z, v.z); v.w = fmaf(p.beta, o.w, v.w);
+            }
+            if (crow) *reinterpret_cast<float4*>(crow + j) = v;
+            if (brow) {
+              const float4 b = make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z),
+                                           tf32_round(v.w));
+              *reinterpret_cast<float4*>(brow + j) = b;
+              *reinterpret_cast<float4*>(srow + j) =
+                  make_float4(v.x - b.x, v.y - b.y, v.z - b.z, v.w - b.w);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < BN; ++j) {
+            if (j < ncol) {
+              float v = p.alpha * acc[j];
+              if (p.beta != 0.f) v = fmaf(p.beta, crow[j], v);
+              if (crow) crow[j] = v;
+              if (brow) {
+                const float b = tf32_round(v);
+                brow[j] = b;
+                srow[j] = v - b;
+              }
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // x -> (tf32(x), x - tf32(x)) for a rows x cols block (row-major, leading dims in elements).
 __global__ void split_tf32_kernel(const float* __restrict__ X, int64_t ldx, int64_t rows,
                                   int64_t cols, float* __restrict__ big, float* __restrict__ small,
@@ -329,10 +558,31 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
   p.vec4 = ((g.C == nullptr || (al16(g.C) && g.ldc % 4 == 0)) &&
             (g.Cbig == nullptr || (al16(g.Cbig) && al16(g.Csmall) && g.ld_split % 4 == 0)))
                ? 1 : 0;
-  const int64_t grid = static_cast<int64_t>(tiles_m) * p.tiles_n;
-  if (grid > 0x7fffffff) return GPTQ_EUNSUPPORTED;
-  gemm_tf32x3_tc<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(tAb, tAs, tBb, tBs,
-                                                                                 p, g.info);
+  p.tiles_m = tiles_m;
+  const bool panel = g.K > 0 && g.K <= tgp::kMaxK && !g.klo_from_m && !g.klo_from_n &&
+                     (!g.lower || g.M == g.N);
+  if (panel) {
+    static bool attr_p = false;
+    if (!attr_p) {
+      if (cudaFuncSetAttribute(gemm_tf32x3_panel_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tgp::kSmemBytes) != cudaSuccess)
+        return GPTQ_ECUDA;
+      attr_p = true;
+    }
+    const int64_t nt = g.lower ? static_cast<int64_t>(tiles_m) * (tiles_m + 1) / 2
+                               : static_cast<int64_t>(tiles_m) * p.tiles_n;
+    if (nt > 0x7fffffff) return GPTQ_EUNSUPPORTED;
+    p.n_tiles = static_cast<int>(nt);
+    const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
+    gemm_tf32x3_panel_tc<<<grid, tgp::kThreads, tgp::kSmemBytes, stream>>>(tAb, tAs, tBb, tBs, p,
+                                                                           g.info);
+  } else {
+    const int64_t grid = static_cast<int64_t>(tiles_m) * p.tiles_n;
+    if (grid > 0x7fffffff) return GPTQ_EUNSUPPORTED;
+    p.n_tiles = static_cast<int>(grid);
+    gemm_tf32x3_tc<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(tAb, tAs, tBb,
+                                                                                   tBs, p, g.info);
+  }
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }

@@ -108,3 +108,16 @@ def test_gemm_lower_tiles_and_k_ranges():
         Vp[i:i + 128, i:i + 128] = np.tril(V[i:i + 128, i:i + 128])
     C, _, _ = _run(T, 0, Vp.T.copy(), 1, klo_n=True)
     _check(C, T, V.T.copy())
+
+
+@pytest.mark.parametrize("n,K", [(384, 128), (1000, 96), (4096, 128)])
+def test_gemm_lower_update_k128(n, K):
+    """The Cholesky trailing update: C -= P P^T on lower tiles, K <= 128 (persistent variant)."""
+    rng = np.random.default_rng(n + K)
+    P = rng.standard_normal((n, K)).astype(np.float32)
+    C0 = rng.standard_normal((n, n)).astype(np.float32)
+    C, _, _ = _run(P, 0, P, 0, alpha=-1.0, beta=1.0, C0=C0, lower=True)
+    tile = np.arange(n) // 128
+    below = tile[:, None] >= tile[None, :]
+    assert np.all(C[~below] == C0[~below])
+    _check(C, P, P, -1.0, 1.0, C0, mask=below)
