@@ -167,30 +167,31 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
     const int c0 = kb * 32;
     if (warp == 0) {
       // lane l owns row c0 + l of the 32 x 32 piece, in registers; the pivot column goes through
-      // shared memory so each step reads it with broadcast loads
+      // shared memory (double-buffered, one warp sync per pivot) so each step reads it with
+      // broadcast loads; pivot reciprocals stay in registers until the piece is done
       float d[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) d[k] = L[(c0 + lane) * LD + c0 + k];
-      float* col = T;  // 32-float scratch
+      float* col = T;  // 2 x 32-float scratch
+      float rr = 0.f;
+      int badj = 32;
 #pragma unroll 32
       for (int j = 0; j < 32; ++j) {
         const float piv = __shfl_sync(0xffffffffu, d[j], j);
         const bool ok = piv > 0.f && piv < INFINITY;
         const float r = ok ? rsqrtf(piv) : 1.f;
-        const float ljj = ok ? piv * r : 1.f;
-        if (lane == 0) {
-          if (!ok && bad < 0) bad = c0 + j;
-          rdiag[c0 + j] = r;
-        }
-        const float a = (lane == j) ? ljj : (lane > j ? d[j] * r : 0.f);
+        badj = (!ok && badj == 32) ? j : badj;
+        rr = (lane == j) ? r : rr;
+        const float a = (lane == j) ? (ok ? piv * r : 1.f) : (lane > j ? d[j] * r : 0.f);
         d[j] = a;
-        col[lane] = a;
+        col[(j & 1) * 32 + lane] = a;
         __syncwarp();
 #pragma unroll 32
         for (int k = 0; k < 32; ++k)
-          if (k > j && lane >= k) d[k] = fmaf(-a, col[k], d[k]);
-        __syncwarp();
+          if (k > j && lane >= k) d[k] = fmaf(-a, col[(j & 1) * 32 + k], d[k]);
       }
+      rdiag[c0 + lane] = rr;
+      if (lane == 0 && badj < 32 && bad < 0) bad = c0 + badj;
 #pragma unroll
       for (int k = 0; k < 32; ++k) L[(c0 + lane) * LD + c0 + k] = (k <= lane) ? d[k] : 0.f;
     }
