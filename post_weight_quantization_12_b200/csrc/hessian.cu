@@ -3,20 +3,22 @@
 // "Part 2: Adaptive Rounding: Optimal Brain Quantizer (OBQ)", section "Goal": the input covariance
 // is the proxy Hessian; "Part 3: Adaptive Rounding: GPTQ", "Algorithm GPTQ": H = X X^T + lambda I.
 //
-// bf16 path: a persistent tcgen05 SYRK. Output is cut into 128 x 256 lower-triangle tiles; each
-// CTA owns one tile per round and walks the whole token range for it, so all CTAs read the same
-// token slab at about the same time (fetched from HBM once, served to the others from L2). Per
-// 32-token stage, TMA brings the 128 channels of the tile's rows (A) and the 256 channels of its
-// columns (B) into shared memory with 128-byte swizzle; both operands are MN-major (channels
-// contiguous), which tcgen05 reads directly, and a tile touching the diagonal reads A out of B's
-// slab. One thread issues two 128 x 256 x 16 MMAs per stage into a TMEM chunk accumulator.
+// bf16 path: a persistent tcgen05 SYRK on CTA pairs (the 2-SM form, cta_group::2). The output is
+// cut into 256 x 256 lower-triangle super-tiles; each pair of CTAs (a cluster of 2 on two SMs) owns
+// one super-tile per round and walks the whole token range for it, so all pairs read the same token
+// slab at about the same time (fetched from HBM once, served to the others from L2). Per 32-token
+// stage each CTA brings, by TMA with 128-byte swizzle, the 128 channels of its half of the rows (A)
+// and of its half of the columns (B) into its own shared memory (16 KB); both operands are MN-major
+// (channels contiguous), which tcgen05 reads directly, and on a diagonal super-tile A doubles as B.
+// The first CTA of the pair issues two 256 x 256 x 16 MMAs per stage; each CTA's TMEM receives its
+// 128 rows. Per SM this moves half the operand bytes of a 128 x 256 single-SM tile.
 //
 // The tensor core adds each MMA's products into its fp32 accumulator with a rounding biased
 // toward zero, so the relative error of one TMEM sum grows with the number of MMAs folded into it
 // (about 6e-8 per MMA measured on B200). Every kChunkStages stages (2048 tokens) the chunk sum is
-// handed to eight epilogue warps, which add it into fp32 registers with IEEE adds while the MMAs
-// fill the other of two chunk buffers (2 x 256 TMEM columns); at the end of the tile the
-// registers are added into S once. Each tile belongs to one CTA: deterministic, no atomics.
+// handed to eight epilogue warps in each CTA, which add it into fp32 registers with IEEE adds while
+// the MMAs fill the other of two chunk buffers (2 x 256 TMEM columns); at the end of the super-tile
+// the registers are added into S once. Each super-tile belongs to one pair: deterministic.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -27,29 +29,18 @@ namespace gptq {
 
 namespace syrk {
 constexpr int kBK = 32;                    // tokens per stage
-constexpr int kStages = 8;
+constexpr int kStages = 12;
 constexpr int kBoxCh = 64;                 // channels per TMA box (128 bytes of bf16)
 constexpr int kBoxBytes = kBoxCh * kBK * 2;          // 4 KB
-constexpr int kABytes = 2 * kBoxBytes;               // 128 channels
-constexpr int kBBytes = 4 * kBoxBytes;               // 256 channels
-constexpr int kStageBytes = kABytes + kBBytes;       // 24 KB
+constexpr int kHalfBytes = 2 * kBoxBytes;            // 128 channels
+constexpr int kStageBytes = 2 * kHalfBytes;          // A half + B half: 16 KB per CTA
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;
-constexpr int kThreads = 320;              // warp 0 TMA, warp 1 MMA, warps 2-9 fold/epilogue
-constexpr uint32_t kTmemCols = 512;        // two 128 x 256 fp32 chunk accumulators
+constexpr int kThreads = 320;              // warp 0 TMA, warp 1 MMA (first CTA), warps 2-9 fold
+constexpr uint32_t kTmemCols = 512;        // two 256-column chunk accumulators (128 rows each)
 constexpr int kChunkStages = 64;           // 2048 tokens per TMEM chunk sum
-constexpr uint32_t kIdesc = make_idesc(/*bf16*/ 1, /*A MN-major*/ 1, /*B MN-major*/ 1, 128, 256);
+constexpr uint32_t kIdesc = make_idesc(/*bf16*/ 1, /*A MN-major*/ 1, /*B MN-major*/ 1, 256, 256);
+constexpr int kEpiWarps = 8;
 }  // namespace syrk
-
-// Lower tiles (I = 128-row block, J = 256-column block, 2J <= I + 1), numbered row-pair by
-// row-pair: rows 2a and 2a+1 each have a+1 tiles.
-__device__ __forceinline__ void decode_tile(int st, int& I, int& J) {
-  int a = static_cast<int>((sqrtf(4.0f * static_cast<float>(st) + 1.0f) - 1.0f) * 0.5f);
-  while ((a + 1) * (a + 2) <= st) ++a;
-  while (a * (a + 1) > st) --a;
-  const int rem = st - a * (a + 1);
-  I = 2 * a + rem / (a + 1);
-  J = rem % (a + 1);
-}
 
 __device__ __forceinline__ void decode_lower(int st, int& I, int& J) {
   int i = static_cast<int>((sqrtf(8.0f * static_cast<float>(st) + 1.0f) - 1.0f) * 0.5f);
@@ -59,23 +50,27 @@ __device__ __forceinline__ void decode_lower(int st, int& I, int& J) {
   J = st - i * (i + 1) / 2;
 }
 
-__global__ void __launch_bounds__(syrk::kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(syrk::kThreads, 1)
 hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ S, int cols,
-                     int n_kblocks, int n_tiles, int32_t* info) {
+                     int n_kblocks, int n_super, int32_t* info) {
   using namespace syrk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
 
-  __shared__ __align__(8) uint64_t full_bar[kStages];
-  __shared__ __align__(8) uint64_t empty_bar[kStages];
-  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
+  __shared__ __align__(8) uint64_t full_bar[kStages];    // used in the first CTA
+  __shared__ __align__(8) uint64_t empty_bar[kStages];   // in both CTAs
+  __shared__ __align__(8) uint64_t acc_full[2];          // in both CTAs
+  __shared__ __align__(8) uint64_t acc_empty[2];         // used in the first CTA
+  __shared__ __align__(8) uint64_t mma_done;             // used in the first CTA
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n_chunks = (n_kblocks + kChunkStages - 1) / kChunkStages;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -84,7 +79,7 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 256);
+      mbar_init(&acc_empty[b], 2 * kEpiWarps);
     }
     mbar_init(&mma_done, 1);
     abort_flag = 0;
@@ -92,56 +87,62 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
     prefetch_tmap(&tmap);
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base_sh, kTmemCols);
-    tmem_relinquish();
+    tmem_alloc_pair(&tmem_base_sh, kTmemCols);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();   // both CTAs' barriers initialised before any cross-CTA signal
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- TMA producer ----------------
+      // ---------------- TMA producer (both CTAs) ----------------
       int s = 0;
       uint32_t ph = 0;
       long long issued = 0;
-      for (int st = blockIdx.x; st < n_tiles && !abort_flag; st += gridDim.x) {
+      for (int st = pair; st < n_super && !abort_flag; st += n_pairs) {
         int I, J;
-        decode_tile(st, I, J);
-        const bool a_in_b = (I >> 1) == J;   // the tile's rows lie inside its column slab
+        decode_lower(st, I, J);
+        const bool diag = (I == J);
+        const uint32_t bytes = diag ? kHalfBytes : kStageBytes;   // this CTA's share
         for (int kb = 0; kb < n_kblocks; ++kb) {
           if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag, info)) goto producer_done;
           uint8_t* a = smem + s * kStageBytes;
-          uint8_t* b = a + kABytes;
-          mbar_arrive_expect_tx(&full_bar[s], a_in_b ? kBBytes : kStageBytes);
+          uint8_t* b = a + kHalfBytes;
+          const uint32_t fb = mapa_shared(smem_u32(&full_bar[s]), 0);
+          if (leader) mbar_arrive_expect_tx(&full_bar[s], 2 * bytes);
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            tma_load_2d(b + q * kBoxBytes, &tmap, &full_bar[s], J * 256 + q * kBoxCh, kb * kBK);
-          if (!a_in_b) {
+          for (int q = 0; q < 2; ++q)
+            tma_load_2d_pair(a + q * kBoxBytes, &tmap, fb,
+                             I * 256 + static_cast<int>(rank) * 128 + q * kBoxCh, kb * kBK);
+          if (!diag) {
 #pragma unroll
             for (int q = 0; q < 2; ++q)
-              tma_load_2d(a + q * kBoxBytes, &tmap, &full_bar[s], I * 128 + q * kBoxCh, kb * kBK);
+              tma_load_2d_pair(b + q * kBoxBytes, &tmap, fb,
+                               J * 256 + static_cast<int>(rank) * 128 + q * kBoxCh, kb * kBK);
           }
           ++issued;
           if (++s == kStages) { s = 0; ph ^= 1u; }
         }
       }
     producer_done:
-      // Let every copy already issued land before the CTA can exit.
-      for (long long i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
-        mbar_drain_bounded(&full_bar[i % kStages], static_cast<uint32_t>((i / kStages) & 1));
+      // the first CTA's full barriers count both CTAs' copies: let every issued copy land
+      if (leader) {
+        for (long long i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+          mbar_drain_bounded(&full_bar[i % kStages], static_cast<uint32_t>((i / kStages) & 1));
+      }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (first CTA of the pair) ----------------
       int s = 0;
       uint32_t ph = 0;
-      int chunk = 0;   // running chunk count: buffer = chunk & 1, its use = chunk >> 1
-      for (int st = blockIdx.x; st < n_tiles && !abort_flag; st += gridDim.x) {
+      int chunk = 0;
+      for (int st = pair; st < n_super && !abort_flag; st += n_pairs) {
         int I, J;
-        decode_tile(st, I, J);
-        const bool a_in_b = (I >> 1) == J;
+        decode_lower(st, I, J);
+        const bool diag = (I == J);
         for (int kc = 0; kc < n_kblocks; kc += kChunkStages, ++chunk) {
           const int buf = chunk & 1;
           if (!mbar_wait_bounded(&acc_empty[buf], ((chunk >> 1) & 1) ^ 1u, &abort_flag, info))
@@ -151,34 +152,36 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
           for (int kb = kc; kb < kc_end; ++kb) {
             if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag, info)) goto mma_done_label;
             tc_fence_after();
-            const uint32_t st_addr = smem_u32(smem + s * kStageBytes);
-            const uint32_t b_addr = st_addr + kABytes;
-            const uint32_t a_addr = a_in_b ? b_addr + (I & 1) * 2 * kBoxBytes : st_addr;
+            const uint32_t a_addr = smem_u32(smem + s * kStageBytes);
+            const uint32_t b_addr = diag ? a_addr : a_addr + kHalfBytes;
 #pragma unroll
             for (int kk = 0; kk < kBK / 16; ++kk) {
               const uint64_t adesc = smem_desc(a_addr + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
               const uint64_t bdesc = smem_desc(b_addr + kk * 2048, kBoxBytes, 1024, kSwizzle128B);
-              tc_mma_f16(tmem + buf * 256, adesc, bdesc, kIdesc, (kb > kc || kk > 0) ? 1u : 0u);
+              tc_mma_f16_pair(tmem + buf * 256, adesc, bdesc, kIdesc,
+                              (kb > kc || kk > 0) ? 1u : 0u);
             }
-            tc_commit(&empty_bar[s]);
+            tc_commit_pair_mc(&empty_bar[s], 0x3);
             if (++s == kStages) { s = 0; ph ^= 1u; }
           }
-          tc_commit(&acc_full[buf]);
+          tc_commit_pair_mc(&acc_full[buf], 0x3);
         }
       }
     mma_done_label:
-      tc_commit(&mma_done);
+      tc_commit_pair(&mma_done);
       mbar_drain_bounded(&mma_done, 0);
     }
   } else {
-    // ---------------- fold chunk sums into registers; add the tile into S at its end ----------
+    // ---------- fold chunk sums into registers; add the super-tile's rows into S at its end ----
     const int q = warp & 3;            // TMEM lane quarter this warp may access
     const int h = (warp - 2) >> 2;     // column half: 0 -> 0..127, 1 -> 128..255
+    const uint32_t ae0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    const uint32_t ae1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
     int chunk = 0;
     bool ok = true;
-    for (int st = blockIdx.x; st < n_tiles && ok && !abort_flag; st += gridDim.x) {
+    for (int st = pair; st < n_super && ok && !abort_flag; st += n_pairs) {
       int I, J;
-      decode_tile(st, I, J);
+      decode_lower(st, I, J);
       float acc[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) acc[j] = 0.f;
@@ -199,10 +202,11 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
           for (int t = 0; t < 32; ++t) acc[cc * 32 + t] += __uint_as_float(v[t]);
         }
         tc_fence_before();
-        mbar_arrive(&acc_empty[buf]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(buf ? ae1 : ae0);
       }
       if (!ok) break;
-      const int i = I * 128 + q * 32 + lane;
+      const int i = I * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
       const int j0 = J * 256 + h * 128;
       if (i < cols) {
         float4* row = reinterpret_cast<float4*>(S + static_cast<size_t>(i) * cols + j0);
@@ -221,11 +225,13 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
     }
   }
 
+  // every MMA of the pair has completed (the first CTA waited for them) before either CTA frees
+  // its tensor memory or exits
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc_pair(tmem, kTmemCols);
   }
 }
 
@@ -299,15 +305,15 @@ gptq_status launch_hessian_bf16(float* S, int64_t cols, const void* X, int64_t n
       return GPTQ_ECUDA;
     attr_done = true;
   }
-  // lower 128 x 256 tiles: row block I has floor(I / 2) + 1 of them
-  const int n_i = static_cast<int>((cols + 127) / 128);
-  int n_tiles = 0;
-  for (int I = 0; I < n_i; ++I) n_tiles += I / 2 + 1;
+  // lower 256 x 256 super-tiles, one per CTA pair per round
+  const int n_s = static_cast<int>((cols + 255) / 256);
+  const int n_super = n_s * (n_s + 1) / 2;
   const int64_t n_kb = (n_tokens + kBK - 1) / kBK;
   if (n_kb > INT32_MAX / kBK) return GPTQ_EUNSUPPORTED;
-  const int grid = n_tiles < num_sms() ? n_tiles : num_sms();
-  hessian_syrk_bf16_tc<<<grid, kThreads, kSmemBytes, stream>>>(
-      tmap, S, static_cast<int>(cols), static_cast<int>(n_kb), n_tiles, info);
+  const int max_pairs = num_sms() / 2;
+  const int pairs = n_super < max_pairs ? n_super : max_pairs;
+  hessian_syrk_bf16_tc<<<2 * pairs, kThreads, kSmemBytes, stream>>>(
+      tmap, S, static_cast<int>(cols), static_cast<int>(n_kb), n_super, info);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }
