@@ -18,6 +18,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 #include "internal.h"
@@ -54,6 +55,7 @@ struct TcGemmParams {
   int tiles_n;
   int vec4;                // C / split rows are 16-byte aligned
   int tiles_m, n_tiles;    // used by the persistent K <= 128 variant
+  int stage_c;             // K <= 128 variant: C goes through shared memory by TMA
 };
 
 // tile index -> (tm, tn): row-major over all tiles, or over the lower triangle tn <= tm
@@ -278,9 +280,15 @@ gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ 
 // ------------------------------------------------------------------------------------------------
 // K <= 128 products (the lazy trailing update, the Cholesky panel solve and trailing update, the
 // triangular inverse's second product): persistent over a contiguous range of output tiles, A and
-// B streamed through two 64 KB stages. Keeping shared memory at 128 KB leaves the rest of the
-// SM's unified L1 to the epilogue, whose row-wise float4 read-modify-write of C (64 KB per tile)
-// then stays in L1; two TMEM buffers let one tile's epilogue overlap the next tile's MMAs.
+// B streamed through two 64 KB stages, two TMEM buffers so one tile's epilogue overlaps the next
+// tile's MMAs.
+//
+// When C is 16-byte addressable the C tile goes through shared memory: four 128-row x 32-column
+// boxes (128-byte swizzle) that one epilogue thread loads by TMA for the next tile as soon as the
+// current tile's store of that box has left shared memory, so the epilogue never waits on a global
+// load; the updated box is written back to shared memory (conflict-free, the swizzle spreads a
+// warp's rows over all banks) and stored by TMA. The tf32 split of the result, when requested, is
+// written straight from registers.
 // ------------------------------------------------------------------------------------------------
 namespace tgp {
 constexpr int BM = 128, BN = 128, BK = 32;
@@ -288,21 +296,24 @@ constexpr int kMaxK = 128;
 constexpr int kPartBytes = BM * BK * 4;             // 16 KB: one part (big or small) of one operand
 constexpr int kStages = 2;
 constexpr int kStageBytes = 4 * kPartBytes;         // A_big, A_small, B_big, B_small
+constexpr int kBoxBytes = BM * 32 * 4;              // 16 KB: 128 rows x 32 columns of C
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;
+constexpr int kSmemBytesStaged = kSmemBytes + 4 * kBoxBytes;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kEpiBarrier = 1;                 // named barrier of the 128 epilogue threads
 }  // namespace tgp
 
 __global__ void __launch_bounds__(tgp::kThreads, 1)
 gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ CUtensorMap tAs,
                      const __grid_constant__ CUtensorMap tBb, const __grid_constant__ CUtensorMap tBs,
-                     TcGemmParams p, int32_t* info) {
+                     const __grid_constant__ CUtensorMap tC, TcGemmParams p, int32_t* info) {
   using namespace tgp;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
-  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done, c_full[4];
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -319,6 +330,7 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
+    for (int j = 0; j < 4; ++j) mbar_init(&c_full[j], 1);
     mbar_init(&mma_done, 1);
     abort_flag = 0;
     fence_mbarrier_init();
@@ -413,6 +425,128 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
     mma_done_label:
       tc_commit(&mma_done);
       mbar_drain_bounded(&mma_done, 0);
+    }
+  } else if (p.stage_c) {
+    // ---- epilogue through shared memory (C loaded and stored by TMA) ----
+    const int q = warp & 3;
+    const int r = q * 32 + lane;                    // row within the tile (= TMEM lane)
+    const uint32_t rsw = static_cast<uint32_t>(r & 7);
+    const bool st_thread = threadIdx.x == 64;       // issues the C loads and stores
+    const bool loads = p.beta != 0.f;
+    uint8_t* cs = smem + kStages * kStageBytes;
+    uint32_t cwait = 0;                             // per-box parity of the next c_full completion
+    uint32_t pend = 0;                              // boxes with a C load in flight (store thread)
+    auto n_boxes = [&](int n0) { return min(4, (p.N - n0 + 31) / 32); };
+    auto load_box = [&](int m0, int n0, int j) {
+      mbar_arrive_expect_tx(&c_full[j], kBoxBytes);
+      tma_load_2d(cs + j * kBoxBytes, &tC, &c_full[j], n0 + 32 * j, m0);
+      pend |= 1u << j;
+    };
+    if (st_thread && loads && t_begin < t_end) {
+      int tm, tn;
+      tile_coords(p, t_begin, tm, tn);
+      const int nbx = n_boxes(tn * BN);
+      for (int j = 0; j < nbx; ++j) load_box(tm * BM, tn * BN, j);
+    }
+    int c = 0;
+    for (int t = t_begin; t < t_end; ++t, ++c) {
+      int tm, tn;
+      tile_coords(p, t, tm, tn);
+      const int m0 = tm * BM, n0 = tn * BN;
+      const int nbx = n_boxes(n0);
+      int nm0 = 0, nn0 = 0, nnb = 0;                // the next tile (nnb = 0: none)
+      if (t + 1 < t_end) {
+        int tm2, tn2;
+        tile_coords(p, t + 1, tm2, tn2);
+        nm0 = tm2 * BM;
+        nn0 = tn2 * BN;
+        nnb = loads ? n_boxes(nn0) : 0;
+      }
+      const int buf = c & 1;
+      const bool ok = mbar_wait_bounded(&acc_full[buf], (c >> 1) & 1, &abort_flag, info);
+      if (named_barrier_or(kEpiBarrier, 128, !ok || abort_flag)) break;
+      tc_fence_after();
+      float acc[BN];
+      const uint32_t t_main = tmem + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t vm[32], vc[32];
+        tmem_ld_32x32b_x32(t_main + cc * 32, vm);
+        tmem_ld_32x32b_x32(t_main + 128 + cc * 32, vc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) acc[cc * 32 + u] = __uint_as_float(vm[u]) + __uint_as_float(vc[u]);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+      const int row = m0 + r;
+      bool stop = false;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (j < nbx && !stop) {
+          bool okc = true;
+          if (loads) {
+            okc = mbar_wait_bounded(&c_full[j], (cwait >> j) & 1u, &abort_flag, info);
+            if (okc) {
+              cwait ^= 1u << j;
+              pend &= ~(1u << j);
+            }
+          }
+          if (okc) {
+            uint8_t* rowp = cs + j * kBoxBytes + r * 128;
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              float4* a = reinterpret_cast<float4*>(rowp + ((static_cast<uint32_t>(u) ^ rsw) << 4));
+              const float* x = acc + j * 32 + 4 * u;
+              float4 v = make_float4(p.alpha * x[0], p.alpha * x[1], p.alpha * x[2], p.alpha * x[3]);
+              if (loads) {
+                const float4 o = *a;
+                v.x = fmaf(p.beta, o.x, v.x); v.y = fmaf(p.beta, o.y, v.y);
+                v.z = fmaf(p.beta, o.z, v.z); v.w = fmaf(p.beta, o.w, v.w);
+              }
+              *a = v;
+              if (p.Cbig && row < p.M) {
+                const int col = n0 + j * 32 + 4 * u;
+                const float4 b = make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z),
+                                             tf32_round(v.w));
+                const float4 sm = make_float4(v.x - b.x, v.y - b.y, v.z - b.z, v.w - b.w);
+                float* bp = p.Cbig + static_cast<int64_t>(row) * p.ld_split + col;
+                float* sp = p.Csmall + static_cast<int64_t>(row) * p.ld_split + col;
+                if (col + 4 <= p.N) {
+                  *reinterpret_cast<float4*>(bp) = b;
+                  *reinterpret_cast<float4*>(sp) = sm;
+                } else {
+                  const float bb[4] = {b.x, b.y, b.z, b.w}, ss[4] = {sm.x, sm.y, sm.z, sm.w};
+                  for (int e = 0; e < 4 && col + e < p.N; ++e) {
+                    bp[e] = bb[e];
+                    sp[e] = ss[e];
+                  }
+                }
+              }
+            }
+          }
+          fence_proxy_async_smem();
+          stop = named_barrier_or(kEpiBarrier, 128, !okc || abort_flag);
+          if (!stop && st_thread) {
+            tma_store_2d(&tC, cs + j * kBoxBytes, n0 + 32 * j, m0);
+            tma_store_commit();
+            if (j >= 1) {
+              tma_store_wait_read<1>();             // box j-1 has left shared memory
+              if (j - 1 < nnb) load_box(nm0, nn0, j - 1);
+            }
+          }
+        }
+      }
+      if (stop) break;
+      if (st_thread) {
+        tma_store_wait_read<0>();
+        for (int j = nbx - 1; j < nnb; ++j) load_box(nm0, nn0, j);
+      }
+    }
+    if (st_thread) {
+      tma_store_wait_all();
+      for (int j = 0; j < 4; ++j)
+        if (pend & (1u << j)) mbar_drain_bounded(&c_full[j], (cwait >> j) & 1u);
     }
   } else {
     const int q = warp & 3;
@@ -559,13 +693,14 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
             (g.Cbig == nullptr || (al16(g.Cbig) && al16(g.Csmall) && g.ld_split % 4 == 0)))
                ? 1 : 0;
   p.tiles_m = tiles_m;
+  p.stage_c = 0;
   const bool panel = g.K > 0 && g.K <= tgp::kMaxK && !g.klo_from_m && !g.klo_from_n &&
                      (!g.lower || g.M == g.N);
   if (panel) {
     static bool attr_p = false;
     if (!attr_p) {
       if (cudaFuncSetAttribute(gemm_tf32x3_panel_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               tgp::kSmemBytes) != cudaSuccess)
+                               tgp::kSmemBytesStaged) != cudaSuccess)
         return GPTQ_ECUDA;
       attr_p = true;
     }
@@ -573,9 +708,17 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
                                : static_cast<int64_t>(tiles_m) * p.tiles_n;
     if (nt > 0x7fffffff) return GPTQ_EUNSUPPORTED;
     p.n_tiles = static_cast<int>(nt);
+    // C through shared memory when a TMA map can describe it (16-byte base and row pitch)
+    CUtensorMap tC;
+    memset(&tC, 0, sizeof(tC));
+    p.stage_c = (g.C != nullptr && p.vec4) ? 1 : 0;
+    if (p.stage_c &&
+        (st = encode_tmap_2d(&tC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.C, 4, g.N, g.M, g.ldc, 32,
+                             tgp::BM, CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK)
+      return st;
     const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
-    gemm_tf32x3_panel_tc<<<grid, tgp::kThreads, tgp::kSmemBytes, stream>>>(tAb, tAs, tBb, tBs, p,
-                                                                           g.info);
+    const int smem = p.stage_c ? tgp::kSmemBytesStaged : tgp::kSmemBytes;
+    gemm_tf32x3_panel_tc<<<grid, tgp::kThreads, smem, stream>>>(tAb, tAs, tBb, tBs, tC, p, g.info);
   } else {
     const int64_t grid = static_cast<int64_t>(tiles_m) * p.tiles_n;
     if (grid > 0x7fffffff) return GPTQ_EUNSUPPORTED;
