@@ -357,13 +357,13 @@ def run_ours(args):
 
     # Per-stage and whole-layer rooflines from the algorithmic work of each stage:
     #   S1: cols*(cols+1)*tokens flop at the bf16 tensor peak;
-    #   S2-S5: 4/3 cols^3 fp32 flop (two Cholesky, one triangular inverse, one triangular
-    #          product), each done as 3 tf32 products: peak = tf32 peak / 3;
+    #   S2-S5: 2/3 cols^3 fp32 flop for the default (reversed) route, one Cholesky and one
+    #          triangular inverse, each done as 3 tf32 products: peak = tf32 peak / 3;
     #   S6-S8: HBM bytes, 9 B per weight for the column loop (read + write fp32, code byte) plus
     #          8 B per trailing element per block for the lazy update (fp32 read + write).
     hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])) * 1e9
     tf32x3 = peak * 1e12 * TF32_PER_BF16 / 3.0
-    fl_25 = 4.0 / 3.0 * cols ** 3
+    fl_25 = 2.0 / 3.0 * cols ** 3
     b_trail = sum(8.0 * rows * (cols - min(cols, b0 + spec.block))
                   for b0 in range(0, cols, spec.block))
     b_68 = 9.0 * rows * cols + b_trail
@@ -393,6 +393,24 @@ def run_ours(args):
     }
     if args.tokens:
         line["note"] = "token count overridden for profiling: not the configured workload"
+
+    # S2-S5 by the pages' three-step route (two Cholesky factorizations, triangular inverse and
+    # product: 4/3 cols^3 flop), timed the same way outside the headline step, for comparison
+    t3 = []
+    for _ in range(3):
+        S.zero_()
+        _lib.hessian_accumulate(S, X, info, stream)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        _lib.prepare_hinv(S, R, n, spec.damp, ws_p, info, stream, route=_lib.GPTQ_ROUTE_THREE_STEP)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        t3.append(a.elapsed_time(b))
+    if int(info.item()) != 0:
+        raise RuntimeError(f"device status {int(info.item())} on the three-step route")
+    line["S2_S5_routes_ms"] = {"reversed (default; the step above)": statistics.mean(s25),
+                               "three_step": statistics.median(t3)}
 
     # end to end through the public API from pinned host buffers
     if not args.no_e2e:

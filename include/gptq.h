@@ -47,10 +47,21 @@ typedef enum gptq_status {
 
 typedef enum gptq_dtype { GPTQ_BF16 = 0, GPTQ_FP32 = 1 } gptq_dtype;
 
+/* How gptq_prepare_hinv_route() reaches R (both give the same R up to rounding: the upper factor
+ * with positive diagonal of (H + lambda I)^-1 is unique). */
+typedef enum gptq_route {
+  GPTQ_ROUTE_DEFAULT = 0,     /* the library's choice: GPTQ_ROUTE_REVERSED */
+  GPTQ_ROUTE_THREE_STEP = 1,  /* Cholesky, triangular inverse, L^-T L^-1, Cholesky of the inverse */
+  GPTQ_ROUTE_REVERSED = 2     /* one Cholesky of the order-reversed matrix, one triangular inverse */
+} gptq_route;
+
 /* Values the kernels write into *info_dev (the first one detected wins). */
 #define GPTQ_INFO_OK 0
-/* 1 .. cols:        H + lambda I is not positive definite; value = 1-based pivot index (S3). */
-/* cols+1 .. 2*cols: the formed inverse is not positive definite; value - cols = pivot (S5). */
+/* 1 .. cols:        H + lambda I is not positive definite; value = 1-based column index of the
+ *                   pivot that failed (S3; for the reversed route the factorization runs from the
+ *                   last column to the first, and the index still names the original column). */
+/* cols+1 .. 2*cols: the formed inverse is not positive definite; value - cols = pivot (S5, three-
+ *                   step route only). */
 #define GPTQ_INFO_TIMEOUT (-1)        /* a bounded wait inside a kernel expired */
 #define GPTQ_INFO_BAD_HESSIAN (-2)    /* mean(diag H) <= 0 or not finite: nothing to damp */
 
@@ -88,8 +99,10 @@ gptq_status gptq_hessian_accumulate(float* S_dev, int64_t cols, const void* X_de
  * (H = 2 X X^T) and "3. Cholesky reformulation" (damping of about 1 % of the mean Hessian
  * diagonal; Cholesky factor computed once); "Part 3: Adaptive Rounding: GPTQ", "Observation 3:
  * The Cholesky Reformulation" and "Algorithm GPTQ" (Cholesky of H^-1, one factor row read per
- * column). The route: H_d = H + lambda I = L L^T (blocked Cholesky), L^-1 (triangular inverse),
- * H_d^-1 = L^-T L^-1, H_d^-1 = R^T R with R upper (Cholesky of the inverse).
+ * column). The pages' route: H_d = H + lambda I = L L^T (blocked Cholesky), L^-1 (triangular
+ * inverse), H_d^-1 = L^-T L^-1, H_d^-1 = R^T R with R upper (Cholesky of the inverse). This call
+ * takes GPTQ_ROUTE_DEFAULT, i.e. the reversed route of gptq_prepare_hinv_route(), which reaches
+ * the same R with half the arithmetic.
  *
  *   S_H_dev    in:  S from gptq_hessian_accumulate (lower triangle read).
  *              out: H = (2 / n_total) S, both triangles, undamped (kept for the layer metric).
@@ -108,6 +121,20 @@ gptq_status gptq_hessian_accumulate(float* S_dev, int64_t cols, const void* X_de
 gptq_status gptq_prepare_hinv(float* S_H_dev, float* R_dev, int64_t cols, int64_t n_total,
                               float damp_rel, void* ws_dev, size_t ws_bytes, int32_t* info_dev,
                               void* stream);
+
+/*
+ * gptq_prepare_hinv with an explicit route (a gptq_route value; anything else is GPTQ_EINVAL).
+ *
+ * GPTQ_ROUTE_THREE_STEP follows the pages step by step (two Cholesky factorizations, a
+ * triangular inverse and a triangular product: 4/3 cols^3 flops). GPTQ_ROUTE_REVERSED uses that
+ * the upper factor is unique: with J the permutation that reverses the column order,
+ * J H_d J = M M^T (lower M) gives H_d = U U^T with U = J M J upper, so H_d^-1 = U^-T U^-1 and
+ * R = U^-1 = J M^-1 J -- one Cholesky and one triangular inverse (2/3 cols^3 flops). Arguments,
+ * outputs, workspace and errors are those of gptq_prepare_hinv.
+ */
+gptq_status gptq_prepare_hinv_route(float* S_H_dev, float* R_dev, int64_t cols, int64_t n_total,
+                                    float damp_rel, int route, void* ws_dev, size_t ws_bytes,
+                                    int32_t* info_dev, void* stream);
 
 /*
  * S6-S8 -- the GPTQ column loop with lazy batch updates.

@@ -18,6 +18,7 @@ GPTQ_BF16, GPTQ_FP32 = 0, 1
 GPTQ_INFO_TIMEOUT = -1
 GPTQ_INFO_BAD_HESSIAN = -2
 GPTQ_WS_PREPARE, GPTQ_WS_QUANTIZE = 1, 2
+GPTQ_ROUTE_DEFAULT, GPTQ_ROUTE_THREE_STEP, GPTQ_ROUTE_REVERSED = 0, 1, 2
 GPTQ_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 
 # name -> (restype, argtypes)
@@ -25,6 +26,7 @@ _P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.
 SIGNATURES = {
     "gptq_hessian_accumulate": (_I32, [_P, _I64, _P, _I32, _I64, _I64, _P, _P]),
     "gptq_prepare_hinv": (_I32, [_P, _P, _I64, _I64, _F, _P, _SZ, _P, _P]),
+    "gptq_prepare_hinv_route": (_I32, [_P, _P, _I64, _I64, _F, _I32, _P, _SZ, _P, _P]),
     "gptq_quantize_layer": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _I32, _I32, _P, _P, _P,
                                    _P, _P, _P, _SZ, _P, _P]),
     "gptq_workspace_size": (_SZ, [_I32, _I64, _I64, _I32]),
@@ -127,11 +129,17 @@ def hessian_accumulate(S, X, info, stream=None):
     _check(st, "gptq_hessian_accumulate")
 
 
-def prepare_hinv(S_H, R, n_total, damp_rel, ws, info, stream=None):
-    """S_H: S in, H = 2S/N out (both triangles); R: upper factor of (H + lambda I)^-1."""
-    st = load().gptq_prepare_hinv(_ptr(S_H), _ptr(R), S_H.shape[0], int(n_total), float(damp_rel),
-                                  _ptr(ws), ws.numel() * ws.element_size(), _ptr(info),
-                                  _stream(stream))
+def prepare_hinv(S_H, R, n_total, damp_rel, ws, info, stream=None, route=None):
+    """S_H: S in, H = 2S/N out (both triangles); R: upper factor of (H + lambda I)^-1.
+
+    route: None for gptq_prepare_hinv (the library's default route), else a GPTQ_ROUTE_* value
+    passed to gptq_prepare_hinv_route."""
+    args = (_ptr(S_H), _ptr(R), S_H.shape[0], int(n_total), float(damp_rel))
+    tail = (_ptr(ws), ws.numel() * ws.element_size(), _ptr(info), _stream(stream))
+    if route is None:
+        st = load().gptq_prepare_hinv(*args, *tail)
+    else:
+        st = load().gptq_prepare_hinv_route(*args, int(route), *tail)
     _check(st, "gptq_prepare_hinv")
 
 

@@ -107,13 +107,22 @@ gptq_status gptq_hessian_accumulate(float* S_dev, int64_t cols, const void* X_de
 gptq_status gptq_prepare_hinv(float* S_H_dev, float* R_dev, int64_t cols, int64_t n_total,
                               float damp_rel, void* ws_dev, size_t ws_bytes, int32_t* info_dev,
                               void* stream) {
+  return gptq_prepare_hinv_route(S_H_dev, R_dev, cols, n_total, damp_rel, GPTQ_ROUTE_DEFAULT,
+                                 ws_dev, ws_bytes, info_dev, stream);
+}
+
+gptq_status gptq_prepare_hinv_route(float* S_H_dev, float* R_dev, int64_t cols, int64_t n_total,
+                                    float damp_rel, int route, void* ws_dev, size_t ws_bytes,
+                                    int32_t* info_dev, void* stream) {
+  if (route != GPTQ_ROUTE_DEFAULT && route != GPTQ_ROUTE_THREE_STEP && route != GPTQ_ROUTE_REVERSED)
+    return GPTQ_EINVAL;
   if (S_H_dev == nullptr || R_dev == nullptr || cols <= 0 || n_total <= 0) return GPTQ_EINVAL;
   if (cols % 4 != 0 || !aligned(S_H_dev, 16) || !aligned(R_dev, 16)) return GPTQ_EINVAL;
   if (!(damp_rel >= 0.f) || !(damp_rel < 1e30f)) return GPTQ_EINVAL;
   if (cols > 65536) return GPTQ_EUNSUPPORTED;
   if (ws_dev == nullptr || ws_bytes < prepare_workspace_bytes(cols) || !aligned(ws_dev, 256))
     return GPTQ_EWORKSPACE;
-  return run_prepare_hinv(S_H_dev, R_dev, cols, n_total, damp_rel, ws_dev, info_dev,
+  return run_prepare_hinv(S_H_dev, R_dev, cols, n_total, damp_rel, route, ws_dev, info_dev,
                           static_cast<cudaStream_t>(stream));
 }
 

@@ -60,7 +60,7 @@ gptq_status launch_split_tf32(const float* X, int64_t ldx, int64_t rows, int64_t
 // S2-S5
 size_t prepare_workspace_bytes(int64_t cols);
 gptq_status run_prepare_hinv(float* S_H, float* R, int64_t cols, int64_t n_total, float damp_rel,
-                             void* ws, int32_t* info, cudaStream_t stream);
+                             int route, void* ws, int32_t* info, cudaStream_t stream);
 
 // S6-S8
 size_t quantize_workspace_bytes(int64_t rows, int64_t cols, int block);

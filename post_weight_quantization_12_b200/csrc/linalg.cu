@@ -5,11 +5,16 @@
 // "Part 3: Adaptive Rounding: GPTQ", "Observation 3" and "Algorithm GPTQ" (Cholesky of H^-1,
 // whose rows are read during quantization).
 //
-// Route: H_d = L L^T (blocked right-looking Cholesky, 128-wide panels), L^-1 (blocked triangular
-// inverse, row block by row block), H_d^-1 = L^-T L^-1 (triangular product, lower half only),
-// H_d^-1 = L2 L2^T (second Cholesky), R = L2^T. Each 128 x 128 diagonal block is factored and
-// inverted on chip by one CTA; everything else is a 3xTF32 tensor-core matrix product whose
-// operands are kept as tf32 (big, small) pairs in the workspace.
+// Two routes to the same R (the upper factor with positive diagonal is unique):
+//  * three-step, as the pages write it: H_d = L L^T (blocked right-looking Cholesky, 128-wide
+//    panels), L^-1 (blocked triangular inverse, row block by row block), H_d^-1 = L^-T L^-1
+//    (triangular product, lower half only), H_d^-1 = L2 L2^T (second Cholesky), R = L2^T;
+//  * reversed: with J the order-reversing permutation, J H_d J = M M^T (one Cholesky), so
+//    H_d = U U^T with U = J M J upper, H_d^-1 = U^-T U^-1 and R = U^-1 = J M^-1 J: one Cholesky
+//    and one triangular inverse, half the flops and half the chain of diagonal blocks.
+// Each 128 x 128 diagonal block is factored and inverted on chip by one CTA; everything else is a
+// 3xTF32 tensor-core matrix product whose operands are kept as tf32 (big, small) pairs in the
+// workspace.
 #include <cmath>
 
 #include "common.cuh"
@@ -120,6 +125,64 @@ __global__ void __launch_bounds__(256) transpose_to_upper_kernel(float* R, int64
   }
 }
 
+// Reversed route: H = (2/N) S mirrored into S_H as above, and the lower triangle of
+// J H_d J (entry [a][b] = H_d[n-1-a][n-1-b]) into R with its strict upper part zeroed.
+__global__ void __launch_bounds__(256)
+finalize_reversed_kernel(float* S_H, float* R, int64_t n, float scale, const float* lam_ptr) {
+  __shared__ float t[32][33];
+  int I, J;
+  decode_tri(blockIdx.x, I, J);
+  const int i0 = I * 32, j0 = J * 32;
+  const float lam = *lam_ptr;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int64_t m = n - 1;
+  for (int r = ty; r < 32; r += 8) {
+    const int i = i0 + r, j = j0 + tx;
+    t[r][tx] = (i < n && j < n) ? S_H[i * n + j] * scale : 0.f;
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    if (I > J) {
+      const int i = i0 + r, j = j0 + tx;
+      if (i < n && j < n) S_H[i * n + j] = t[r][tx];
+      const int it = j0 + r, jt = i0 + tx;          // transposed position (upper tile of H)
+      if (it < n && jt < n) {
+        S_H[it * n + jt] = t[tx][r];
+        R[(m - it) * n + (m - jt)] = t[tx][r];      // H[jt][it], now below the diagonal
+      }
+      if (i < n && j < n) R[(m - i) * n + (m - j)] = 0.f;
+    } else {
+      const int i = i0 + r, j = j0 + tx;
+      if (i < n && j < n) {
+        const float h = (tx <= r) ? t[r][tx] : t[tx][r];
+        S_H[i * n + j] = h;
+        R[(m - i) * n + (m - j)] = (tx > r) ? h : (tx == r ? h + lam : 0.f);
+      }
+    }
+  }
+}
+
+// Reversed route, last step: R = J V J with V = (Vb + Vs) the lower triangular inverse (ld n);
+// the result is upper, its strict lower part zeroed. One lower 32 x 32 tile of V per CTA.
+__global__ void __launch_bounds__(256)
+reverse_to_upper_kernel(float* R, const float* Vb, const float* Vs, int64_t n) {
+  int I, J;
+  decode_tri(blockIdx.x, I, J);
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int64_t m = n - 1;
+  for (int r = ty; r < 32; r += 8) {
+    const int a = I * 32 + r, b = J * 32 + tx;
+    if (a < n && b < n) {
+      const float v = (a >= b) ? Vb[a * n + b] + Vs[a * n + b] : 0.f;
+      R[(m - a) * n + (m - b)] = v;
+    }
+    if (I > J) {                                    // the mirrored tile lands below the diagonal
+      const int a2 = J * 32 + r, b2 = I * 32 + tx;
+      if (a2 < n && b2 < n) R[(m - a2) * n + (m - b2)] = 0.f;
+    }
+  }
+}
+
 // ------------------------------------------------------------------------------------------------
 // S3/S5 diagonal block: Cholesky of A[k0:k0+nb, k0:k0+nb] on chip (lower; the block's strict upper
 // part is zeroed in A) and the tf32 split of its triangular inverse into (Db, Ds) with ld ldd.
@@ -128,11 +191,13 @@ __global__ void __launch_bounds__(256) transpose_to_upper_kernel(float* R, int64
 // inverts the piece while warps 1-3 solve the rows below it by forward substitution; all warps
 // update the trailing part. The off-diagonal pieces of the inverse follow from
 // X[bi][bj] = -X[bi][bi] * sum_k L[bi][k] X[k][bj]. A pivot that is not positive records
-// info_base + k0 + j + 1 and is replaced by 1 so the remaining arithmetic stays finite.
+// info_base + k0 + j + 1 (or, for a factorization of the order-reversed matrix of order rev_n > 0,
+// the 1-based index of that pivot in the original order, rev_n - k0 - j) and is replaced by 1 so
+// the remaining arithmetic stays finite.
 // ------------------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(la::kDiagThreads)
 potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, int64_t ldd,
-                  int32_t* info, int info_base) {
+                  int32_t* info, int info_base, int rev_n) {
   constexpr int NB = 128, LD = 129;
   extern __shared__ float sm[];
   float* L = sm;
@@ -271,7 +336,8 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
     }
     __syncthreads();
   }
-  if (tid == 0 && bad >= 0 && bad < nb) record_info(info, info_base + k0 + bad + 1);
+  if (tid == 0 && bad >= 0 && bad < nb)
+    record_info(info, rev_n > 0 ? rev_n - (k0 + bad) : info_base + k0 + bad + 1);
   // off-diagonal pieces of the inverse, 2 x 2 outputs per thread (rows r, r+16; cols c, c+16)
   for (int bi = 1; bi < 4; ++bi) {
     for (int e = tid; e < bi * 256; e += 512) {
@@ -339,7 +405,7 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
 }
 
 static gptq_status launch_potrf_diag(float* A, int64_t n, int k0, int nb, float* Db, float* Ds,
-                                     int64_t ldd, int32_t* info, int info_base,
+                                     int64_t ldd, int32_t* info, int info_base, int rev_n,
                                      cudaStream_t stream) {
   static bool attr_done = false;
   if (!attr_done) {
@@ -349,7 +415,7 @@ static gptq_status launch_potrf_diag(float* A, int64_t n, int k0, int nb, float*
     attr_done = true;
   }
   potrf_diag_kernel<<<1, la::kDiagThreads, la::kDiagSmem, stream>>>(A, n, k0, nb, Db, Ds, ldd, info,
-                                                                     info_base);
+                                                                     info_base, rev_n);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }
@@ -363,16 +429,17 @@ struct Split {
 //   Lsp:  tf32 split of L's panels (n x n, ld n), written as the panels are solved;
 //   Dsp:  where each diagonal block's inverse goes (ld ld_dinv): at block k0 of an n x n matrix
 //         when per_block is set (the block diagonal of L^-1), else one shared 128 x 128 scratch;
-//   Psp:  split of the current panel before its solve (n x 128).
+//   Psp:  split of the current panel before its solve (n x 128);
+//   rev_n: > 0 when A is the order-reversed matrix (pivot codes then name original columns).
 static gptq_status potrf_blocked(float* A, int64_t n, Split Lsp, Split Dsp, int64_t ld_dinv,
                                  bool per_block, Split Psp, int32_t* info, int info_base,
-                                 cudaStream_t stream) {
+                                 int rev_n, cudaStream_t stream) {
   using namespace la;
   for (int64_t k0 = 0; k0 < n; k0 += kNB) {
     const int nb = static_cast<int>(n - k0 < kNB ? n - k0 : kNB);
     const int64_t doff = per_block ? k0 * ld_dinv + k0 : 0;
     GPTQ_TRY(launch_potrf_diag(A, n, static_cast<int>(k0), nb, Dsp.b + doff, Dsp.s + doff, ld_dinv,
-                               info, info_base, stream));
+                               info, info_base, rev_n, stream));
     const int64_t m = n - k0 - nb;
     if (m == 0) break;
     float* A21 = A + (k0 + nb) * n + k0;
@@ -425,7 +492,7 @@ size_t prepare_workspace_bytes(int64_t cols) {
 }
 
 gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, float damp_rel,
-                             void* ws, int32_t* info, cudaStream_t stream) {
+                             int route, void* ws, int32_t* info, cudaStream_t stream) {
   using namespace la;
   PrepareWs w = carve(ws, n);
 
@@ -436,12 +503,19 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
   if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
   const int nt = static_cast<int>((n + 31) / 32);
   const int ntri = nt * (nt + 1) / 2;
-  finalize_kernel<<<ntri, dim3(32, 8), 0, stream>>>(S_H, R, n, static_cast<float>(scale), w.lam);
+  const bool reversed = route != GPTQ_ROUTE_THREE_STEP;
+  if (reversed)
+    finalize_reversed_kernel<<<ntri, dim3(32, 8), 0, stream>>>(S_H, R, n, static_cast<float>(scale),
+                                                               w.lam);
+  else
+    finalize_kernel<<<ntri, dim3(32, 8), 0, stream>>>(S_H, R, n, static_cast<float>(scale), w.lam);
   count_launch();
   if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
 
-  // S3: H_d = L L^T in R; the inverses of L's diagonal blocks land in V (the split of L^-1)
-  GPTQ_TRY(potrf_blocked(R, n, w.L, w.V, n, true, w.P, info, 0, stream));
+  // S3: H_d = L L^T in R (reversed route: J H_d J = M M^T, M written as L below); the inverses of
+  // L's diagonal blocks land in V (the split of L^-1)
+  GPTQ_TRY(potrf_blocked(R, n, w.L, w.V, n, true, w.P, info, 0, reversed ? static_cast<int>(n) : 0,
+                         stream));
 
   // S4a: the rest of L^-1, row block by row block:
   //   T = L[i, :i] * Linv[:i, :i];  Linv[i, :i] = -Linv[i, i] * T
@@ -457,6 +531,13 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
     GPTQ_TRY(launch_gemm_tc(u, stream));
   }
 
+  if (reversed) {
+    // R = J M^-1 J
+    reverse_to_upper_kernel<<<ntri, dim3(32, 8), 0, stream>>>(R, w.V.b, w.V.s, n);
+    count_launch();
+    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+  }
+
   // S4b: H_d^-1 = L^-T L^-1 (lower tiles) into R
   TcGemmArgs h{w.V.b, w.V.s, w.V.b, w.V.s, n, n, 1, 1,
                static_cast<int>(n), static_cast<int>(n), static_cast<int>(n), 1.f, 0.f, 1, 1, 0,
@@ -464,7 +545,7 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
   GPTQ_TRY(launch_gemm_tc(h, stream));
 
   // S5: H_d^-1 = L2 L2^T (reusing the L split and the diagonal scratch), then R = L2^T
-  GPTQ_TRY(potrf_blocked(R, n, w.L, w.D, kNB, false, w.P, info, static_cast<int>(n), stream));
+  GPTQ_TRY(potrf_blocked(R, n, w.L, w.D, kNB, false, w.P, info, static_cast<int>(n), 0, stream));
   transpose_to_upper_kernel<<<ntri, dim3(32, 8), 0, stream>>>(R, n);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;

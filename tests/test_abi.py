@@ -79,6 +79,11 @@ def test_other_entry_points_reject_bad_arguments(built_lib):
         _lib.GPTQ_EINVAL
     assert lib.gptq_prepare_hinv(FAKE, FAKE, 128, 10, 0.01, FAKE, 16, FAKE, None) == \
         _lib.GPTQ_EWORKSPACE
+    for route in (-1, 3):
+        assert lib.gptq_prepare_hinv_route(FAKE, FAKE, 128, 10, 0.01, route, FAKE, 1 << 30, FAKE,
+                                           None) == _lib.GPTQ_EINVAL
+    assert lib.gptq_prepare_hinv_route(FAKE, FAKE, 128, 10, 0.01, _lib.GPTQ_ROUTE_REVERSED, FAKE,
+                                       16, FAKE, None) == _lib.GPTQ_EWORKSPACE
     st = lib.gptq_quantize_layer(FAKE, _lib.GPTQ_FP32, 64, 128, 128, FAKE, 4, -1, 32, FAKE, FAKE,
                                  FAKE, FAKE, None, FAKE, 16, FAKE, None)
     assert st == _lib.GPTQ_EWORKSPACE

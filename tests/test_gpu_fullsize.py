@@ -25,12 +25,14 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda"
 
 CASES = {
-    # name: (spec, rows sampled, oracle columns (None = all), trailing block for R)
-    "attn_4096x4096": (synth.ATTN, 24, None, 1024),
-    "mlp_up_11008x4096": (synth.MLP_UP, 16, None, 1024),
-    "mlp_down_4096x11008": (synth.MLP_DOWN, 12, None, 1536),
-    "fc1_49152x12288_3bit_row": (dataclasses.replace(synth.FC1, bits=3, group=-1), 8, None, 1536),
-    "fc2_12288x49152_4bit_g128": (synth.FC2, 16, 1024, 1024),
+    # name: (spec, rows sampled, oracle columns (None = all), trailing block for R, route)
+    "attn_4096x4096": (synth.ATTN, 24, None, 1024, None),
+    "attn_4096x4096_three_step": (synth.ATTN, 24, None, 1024, _lib.GPTQ_ROUTE_THREE_STEP),
+    "mlp_up_11008x4096": (synth.MLP_UP, 16, None, 1024, None),
+    "mlp_down_4096x11008": (synth.MLP_DOWN, 12, None, 1536, None),
+    "fc1_49152x12288_3bit_row": (dataclasses.replace(synth.FC1, bits=3, group=-1), 8, None, 1536,
+                                 None),
+    "fc2_12288x49152_4bit_g128": (synth.FC2, 16, 1024, 1024, None),
 }
 
 
@@ -40,7 +42,7 @@ def _rel_fro(a, b):
 
 @pytest.mark.parametrize("name", list(CASES))
 def test_full_size_against_sampled_oracle(name):
-    spec, n_rows, ocols, tb = CASES[name]
+    spec, n_rows, ocols, tb, route = CASES[name]
     seed = 0
     free = torch.cuda.mem_get_info()[0]
     need = spec.n_tokens * spec.cols * 2 + 6 * spec.cols ** 2 * 4 + 12 * spec.rows * spec.cols
@@ -68,7 +70,7 @@ def test_full_size_against_sampled_oracle(name):
     R = torch.empty(cols, cols, device=DEV)
     ws = torch.empty(_lib.workspace_size(_lib.GPTQ_WS_PREPARE, 0, cols, 0), dtype=torch.uint8,
                      device=DEV)
-    _lib.prepare_hinv(S, R, n, spec.damp, ws, info)
+    _lib.prepare_hinv(S, R, n, spec.damp, ws, info, route=route)
     torch.cuda.synchronize()
     assert info.item() == 0
     del ws

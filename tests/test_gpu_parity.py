@@ -44,13 +44,13 @@ def gpu_hessian(X_np, x_dtype, chunks=1):
     return S
 
 
-def gpu_prepare(S, n_total, damp=0.01):
+def gpu_prepare(S, n_total, damp=0.01, route=None):
     cols = S.shape[0]
     R = torch.empty(cols, cols, device=DEV)
     ws = torch.empty(_lib.workspace_size(_lib.GPTQ_WS_PREPARE, 0, cols, 0), dtype=torch.uint8,
                      device=DEV)
     info = new_info()
-    _lib.prepare_hinv(S, R, n_total, damp, ws, info)
+    _lib.prepare_hinv(S, R, n_total, damp, ws, info, route=route)
     torch.cuda.synchronize()
     return R, int(info.item())
 
@@ -106,13 +106,17 @@ def test_hessian_bf16_tensor_cores(cols, n_tokens, chunks):
 # S2-S5
 # ------------------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("cols,n_tokens", [(128, 1024), (300, 2048), (1024, 8192)])
-def test_prepare_hinv_stagewise(cols, n_tokens):
+ROUTES = [None, _lib.GPTQ_ROUTE_THREE_STEP, _lib.GPTQ_ROUTE_REVERSED]
+
+
+@pytest.mark.parametrize("route", ROUTES, ids=["default", "three_step", "reversed"])
+@pytest.mark.parametrize("cols,n_tokens", [(128, 1024), (300, 2048), (1024, 8192), (644, 4096)])
+def test_prepare_hinv_stagewise(cols, n_tokens, route):
     spec = synth.scaled_spec(synth.ATTN, 8, cols, n_tokens, x_dtype="fp32")
     X = synth.inputs_np(spec, 2)
     S = gpu_hessian(X, torch.float32)
     S_in = S.cpu().numpy().astype(np.float64)
-    R, info = gpu_prepare(S, n_tokens)
+    R, info = gpu_prepare(S, n_tokens, route=route)
     assert info == 0
     H_gpu = S.cpu().numpy()
     H_ref = oracle.hessian_finalize(np.tril(S_in) + np.tril(S_in, -1).T, n_tokens)
@@ -124,12 +128,13 @@ def test_prepare_hinv_stagewise(cols, n_tokens):
     assert rel_fro(R_gpu, R_ref) < 1e-4
 
 
-def test_prepare_reports_non_pd_pivot():
+@pytest.mark.parametrize("route", ROUTES, ids=["default", "three_step", "reversed"])
+def test_prepare_reports_non_pd_pivot(route):
     cols = 256
     S = torch.eye(cols, device=DEV) * 50.0
     S[37, 37] = -1.0e4          # after damping this pivot stays negative
-    _, info = gpu_prepare(S, 100)
-    assert info == 38
+    _, info = gpu_prepare(S, 100, route=route)
+    assert info == 38           # the original column, whichever order the factorization runs in
     assert _lib.info_status(info) == _lib.GPTQ_ENOTPD
 
 
