@@ -56,6 +56,8 @@ struct TcGemmParams {
   int vec4;                // C / split rows are 16-byte aligned
   int tiles_m, n_tiles;    // used by the persistent K <= 128 variant
   int stage_c;             // K <= 128 variant: C goes through shared memory by TMA
+  int khi_from_m;
+  int bstride;             // diagonal shift between batches (elements)
 };
 
 // tile index -> (tm, tn): row-major over all tiles, or over the lower triangle tn <= tm
@@ -77,13 +79,17 @@ gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ 
                const __grid_constant__ CUtensorMap tBb, const __grid_constant__ CUtensorMap tBs,
                TcGemmParams p, int32_t* info) {
   using namespace tg;
-  const int tm = blockIdx.x / p.tiles_n, tn = blockIdx.x % p.tiles_n;
+  const int per_batch = p.tiles_m * p.tiles_n;
+  const int bt = blockIdx.x / per_batch, tix = blockIdx.x - bt * per_batch;
+  const int tm = tix / p.tiles_n, tn = tix - (tix / p.tiles_n) * p.tiles_n;
   const int m0 = tm * BM, n0 = tn * BN;
+  const int boff = bt * p.bstride;          // this batch's shift along the diagonal
   if (p.lower && n0 > m0 + BM - 1) return;  // tile entirely above the diagonal
   int klo = 0;
   if (p.klo_from_m) klo = max(klo, m0);
   if (p.klo_from_n) klo = max(klo, n0);
-  const int nk = p.K > klo ? (p.K - klo + BK - 1) / BK : 0;
+  const int khi = p.khi_from_m ? min(p.K, m0 + BM) : p.K;
+  const int nk = khi > klo ? (khi - klo + BK - 1) / BK : 0;
   const int n_chunks = (nk + kChunkStages - 1) / kChunkStages;
 
   extern __shared__ uint8_t smem_raw[];
@@ -125,28 +131,29 @@ gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ 
       for (int kb = 0; kb < nk; ++kb) {
         if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag, info)) break;
         uint8_t* st = smem + s * kStageBytes;
-        const int k0 = klo + kb * BK;
+        const int k0 = klo + kb * BK + boff;
+        const int am = m0 + boff, bn = n0 + boff;
         mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
         // A parts at st + 0 / kOpBytes, B parts at st + 2 / 3 * kOpBytes
         if (p.a_mn) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            tma_load_2d(st + q * 4096, &tAb, &full_bar[s], m0 + 32 * q, k0);
-            tma_load_2d(st + kOpBytes + q * 4096, &tAs, &full_bar[s], m0 + 32 * q, k0);
+            tma_load_2d(st + q * 4096, &tAb, &full_bar[s], am + 32 * q, k0);
+            tma_load_2d(st + kOpBytes + q * 4096, &tAs, &full_bar[s], am + 32 * q, k0);
           }
         } else {
-          tma_load_2d(st, &tAb, &full_bar[s], k0, m0);
-          tma_load_2d(st + kOpBytes, &tAs, &full_bar[s], k0, m0);
+          tma_load_2d(st, &tAb, &full_bar[s], k0, am);
+          tma_load_2d(st + kOpBytes, &tAs, &full_bar[s], k0, am);
         }
         if (p.b_mn) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            tma_load_2d(st + 2 * kOpBytes + q * 4096, &tBb, &full_bar[s], n0 + 32 * q, k0);
-            tma_load_2d(st + 3 * kOpBytes + q * 4096, &tBs, &full_bar[s], n0 + 32 * q, k0);
+            tma_load_2d(st + 2 * kOpBytes + q * 4096, &tBb, &full_bar[s], bn + 32 * q, k0);
+            tma_load_2d(st + 3 * kOpBytes + q * 4096, &tBs, &full_bar[s], bn + 32 * q, k0);
           }
         } else {
-          tma_load_2d(st + 2 * kOpBytes, &tBb, &full_bar[s], k0, n0);
-          tma_load_2d(st + 3 * kOpBytes, &tBs, &full_bar[s], k0, n0);
+          tma_load_2d(st + 2 * kOpBytes, &tBb, &full_bar[s], k0, bn);
+          tma_load_2d(st + 3 * kOpBytes, &tBs, &full_bar[s], k0, bn);
         }
         ++issued;
         if (++s == kStages) { s = 0; ph ^= 1u; }
@@ -228,9 +235,10 @@ gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ 
       mbar_arrive(&acc_empty[buf]);
     }
     if (ok && row < p.M) {
-      float* crow = p.C ? p.C + static_cast<int64_t>(row) * p.ldc + n0 : nullptr;
-      float* brow = p.Cbig ? p.Cbig + static_cast<int64_t>(row) * p.ld_split + n0 : nullptr;
-      float* srow = p.Cbig ? p.Csmall + static_cast<int64_t>(row) * p.ld_split + n0 : nullptr;
+      const int64_t grow = row + boff, gcol = n0 + boff;
+      float* crow = p.C ? p.C + grow * p.ldc + gcol : nullptr;
+      float* brow = p.Cbig ? p.Cbig + grow * p.ld_split + gcol : nullptr;
+      float* srow = p.Cbig ? p.Csmall + grow * p.ld_split + gcol : nullptr;
       const int ncol = min(BN, p.N - n0);
       if (p.vec4 && ncol == BN) {
 #pragma unroll
@@ -663,16 +671,19 @@ static bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) 
 
 gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
   using namespace tg;
-  if (g.M <= 0 || g.N <= 0) return GPTQ_OK;
+  if (g.M <= 0 || g.N <= 0 || g.batch <= 0) return GPTQ_OK;
   if (!al16(g.Ab) || !al16(g.As) || !al16(g.Bb) || !al16(g.Bs) || g.lda % 4 || g.ldb % 4)
     return GPTQ_EINVAL;
+  if (g.batch > 1 && (g.bstride <= 0 || g.bstride % 4 || g.bstride > (1 << 24))) return GPTQ_EINVAL;
   const int K = g.K > 0 ? g.K : 1;  // an empty K still needs valid maps
+  // the maps span every batch: batch b reads rows/columns shifted by b * bstride
+  const int64_t ext = g.batch > 1 ? (g.batch - 1) * g.bstride : 0;
   CUtensorMap tAb, tAs, tBb, tBs;
   gptq_status st;
-  if ((st = operand_map(&tAb, g.Ab, g.lda, g.a_mn, g.M, K)) != GPTQ_OK) return st;
-  if ((st = operand_map(&tAs, g.As, g.lda, g.a_mn, g.M, K)) != GPTQ_OK) return st;
-  if ((st = operand_map(&tBb, g.Bb, g.ldb, g.b_mn, g.N, K)) != GPTQ_OK) return st;
-  if ((st = operand_map(&tBs, g.Bs, g.ldb, g.b_mn, g.N, K)) != GPTQ_OK) return st;
+  if ((st = operand_map(&tAb, g.Ab, g.lda, g.a_mn, g.M + ext, K + ext)) != GPTQ_OK) return st;
+  if ((st = operand_map(&tAs, g.As, g.lda, g.a_mn, g.M + ext, K + ext)) != GPTQ_OK) return st;
+  if ((st = operand_map(&tBb, g.Bb, g.ldb, g.b_mn, g.N + ext, K + ext)) != GPTQ_OK) return st;
+  if ((st = operand_map(&tBs, g.Bs, g.ldb, g.b_mn, g.N + ext, K + ext)) != GPTQ_OK) return st;
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(gemm_tf32x3_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -694,8 +705,10 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
                ? 1 : 0;
   p.tiles_m = tiles_m;
   p.stage_c = 0;
+  p.khi_from_m = g.khi_from_m;
+  p.bstride = static_cast<int>(g.batch > 1 ? g.bstride : 0);
   const bool panel = g.K > 0 && g.K <= tgp::kMaxK && !g.klo_from_m && !g.klo_from_n &&
-                     (!g.lower || g.M == g.N);
+                     !g.khi_from_m && g.batch == 1 && (!g.lower || g.M == g.N);
   if (panel) {
     static bool attr_p = false;
     if (!attr_p) {
@@ -720,7 +733,7 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
     const int smem = p.stage_c ? tgp::kSmemBytesStaged : tgp::kSmemBytes;
     gemm_tf32x3_panel_tc<<<grid, tgp::kThreads, smem, stream>>>(tAb, tAs, tBb, tBs, tC, p, g.info);
   } else {
-    const int64_t grid = static_cast<int64_t>(tiles_m) * p.tiles_n;
+    const int64_t grid = static_cast<int64_t>(tiles_m) * p.tiles_n * g.batch;
     if (grid > 0x7fffffff) return GPTQ_EUNSUPPORTED;
     p.n_tiles = static_cast<int>(grid);
     gemm_tf32x3_tc<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(tAb, tAs, tBb,

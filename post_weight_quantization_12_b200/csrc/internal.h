@@ -30,9 +30,13 @@ gptq_status launch_hessian_f32(float* S, int64_t cols, const float* X, int64_t n
 //   opA[m][k] = a_mn ? A[k * lda + m] : A[m * lda + k]
 //   opB[k][n] = b_mn ? B[k * ldb + n] : B[n * ldb + k]
 // With `lower`, 128 x 128 output tiles entirely above the diagonal m == n are skipped.
-// klo = max(0, m0 if klo_from_m, n0 if klo_from_n) for the tile's first row m0 / column n0, to
-// skip known-zero triangles (m0, n0 are multiples of 128). C may be null (then beta must be 0);
-// if Cbig is set, the tf32 split of the result is also written there (ld_split).
+// klo = max(0, m0 if klo_from_m, n0 if klo_from_n) for the tile's first row m0 / column n0, and
+// khi = min(K, m0 + 128 if khi_from_m), to skip known-zero triangles (m0, n0 are multiples of
+// 128). C may be null (then beta must be 0); if Cbig is set, the tf32 split of the result is also
+// written there (ld_split).
+// Batches: `batch` independent products of the same shape whose operands and results sit
+// bstride rows and bstride columns further along the same matrices (blocks along a diagonal);
+// every coordinate of A, B, C and the split is shifted by b * bstride for batch b.
 // Requirements: operand bases 16-byte aligned, lda % 4 == 0, ldb % 4 == 0.
 struct TcGemmArgs {
   const float* Ab;
@@ -50,6 +54,9 @@ struct TcGemmArgs {
   float* Csmall;
   int64_t ld_split;
   int32_t* info;
+  int batch = 1;
+  int64_t bstride = 0;
+  int khi_from_m = 0;
 };
 gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream);
 

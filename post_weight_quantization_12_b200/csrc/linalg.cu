@@ -461,7 +461,7 @@ static gptq_status potrf_blocked(float* A, int64_t n, Split Lsp, Split Dsp, int6
 
 namespace {
 struct PrepareWs {
-  Split L, V, P, T, D;
+  Split L, V, P, D;
   float* lam;
 };
 
@@ -478,16 +478,55 @@ PrepareWs carve(void* ws, int64_t n) {
   w.L.b = take(nn); w.L.s = take(nn);
   w.V.b = take(nn); w.V.s = take(nn);
   w.P.b = take(np); w.P.s = take(np);
-  w.T.b = take(np); w.T.s = take(np);
   w.D.b = take(kNB * kNB * 4); w.D.s = take(kNB * kNB * 4);
   w.lam = take(256);
   return w;
 }
 }  // namespace
 
+// S4a: L^-1 (into the split V, whose 128 x 128 diagonal blocks already hold the inverses of L's
+// diagonal blocks) by recursive doubling. For a diagonal block of size s1 + s2 split into halves,
+//   [L11 0; L21 L22]^-1 = [V11 0; V21 V22],  V21 = -V22 (L21 V11),
+// so once every block of size s is inverted, all blocks of size 2s follow from two batched
+// products (all merges of one level at once; a last, shorter merge separately):
+//   T^T = V11^T L21^T   (s x s2; V11 lower, so k starts at the tile's row),
+//   V21 = -V22 T         (s2 x s; V22 lower, so k stops after the tile's rows).
+// T^T is kept in V's strict upper triangle at [o : o+s, o+s : o+s+s2], which nothing else reads.
+static gptq_status trtri_merge(const PrepareWs& w, int64_t n, int64_t o, int64_t s1, int64_t s2,
+                               int batch, int32_t* info, cudaStream_t stream) {
+  const int64_t t_off = o * n + o + s1;               // T^T block
+  const int64_t v21_off = (o + s1) * n + o;           // V21 block
+  TcGemmArgs t{w.V.b + o * n + o, w.V.s + o * n + o, w.L.b + (o + s1) * n + o,
+               w.L.s + (o + s1) * n + o, n, n, 1, 0,
+               static_cast<int>(s1), static_cast<int>(s2), static_cast<int>(s1), 1.f, 0.f, 0, 1, 0,
+               nullptr, 0, w.V.b + t_off, w.V.s + t_off, n, info};
+  t.batch = batch;
+  t.bstride = 2 * s1;
+  GPTQ_TRY(launch_gemm_tc(t, stream));
+  TcGemmArgs u{w.V.b + (o + s1) * n + o + s1, w.V.s + (o + s1) * n + o + s1, w.V.b + t_off,
+               w.V.s + t_off, n, n, 0, 0,
+               static_cast<int>(s2), static_cast<int>(s1), static_cast<int>(s2), -1.f, 0.f, 0, 0, 0,
+               nullptr, 0, w.V.b + v21_off, w.V.s + v21_off, n, info};
+  u.batch = batch;
+  u.bstride = 2 * s1;
+  u.khi_from_m = 1;
+  return launch_gemm_tc(u, stream);
+}
+
+static gptq_status trtri_doubling(const PrepareWs& w, int64_t n, int32_t* info,
+                                  cudaStream_t stream) {
+  for (int64_t s = la::kNB; s < n; s *= 2) {
+    const int64_t full = n / (2 * s);                 // merges whose halves are both s wide
+    if (full > 0) GPTQ_TRY(trtri_merge(w, n, 0, s, s, static_cast<int>(full), info, stream));
+    const int64_t o = full * 2 * s;
+    if (o + s < n) GPTQ_TRY(trtri_merge(w, n, o, s, n - o - s, 1, info, stream));
+  }
+  return GPTQ_OK;
+}
+
 size_t prepare_workspace_bytes(int64_t cols) {
   const size_t n = static_cast<size_t>(cols);
-  return 4 * align_up(n * n * 4, 256) + 4 * align_up(n * la::kNB * 4, 256) +
+  return 4 * align_up(n * n * 4, 256) + 2 * align_up(n * la::kNB * 4, 256) +
          2 * align_up(la::kNB * la::kNB * 4, 256) + 256;
 }
 
@@ -517,19 +556,8 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
   GPTQ_TRY(potrf_blocked(R, n, w.L, w.V, n, true, w.P, info, 0, reversed ? static_cast<int>(n) : 0,
                          stream));
 
-  // S4a: the rest of L^-1, row block by row block:
-  //   T = L[i, :i] * Linv[:i, :i];  Linv[i, :i] = -Linv[i, i] * T
-  for (int64_t r0 = kNB; r0 < n; r0 += kNB) {
-    const int rb = static_cast<int>(n - r0 < kNB ? n - r0 : kNB);
-    TcGemmArgs t{w.L.b + r0 * n, w.L.s + r0 * n, w.V.b, w.V.s, n, n, 0, 1,
-                 rb, static_cast<int>(r0), static_cast<int>(r0), 1.f, 0.f, 0, 0, 1,
-                 nullptr, 0, w.T.b, w.T.s, n, info};
-    GPTQ_TRY(launch_gemm_tc(t, stream));
-    TcGemmArgs u{w.V.b + r0 * n + r0, w.V.s + r0 * n + r0, w.T.b, w.T.s, n, n, 0, 1,
-                 rb, static_cast<int>(r0), rb, -1.f, 0.f, 0, 0, 0,
-                 nullptr, 0, w.V.b + r0 * n, w.V.s + r0 * n, n, info};
-    GPTQ_TRY(launch_gemm_tc(u, stream));
-  }
+  // S4a: the rest of L^-1 by recursive doubling over the diagonal blocks already inverted.
+  GPTQ_TRY(trtri_doubling(w, n, info, stream));
 
   if (reversed) {
     // R = J M^-1 J
