@@ -26,7 +26,7 @@ namespace la {
 constexpr int kNB = 128;       // panel / diagonal block width
 constexpr int kLd = kNB + 1;   // padded shared-memory row
 constexpr int kDiagThreads = 512;
-constexpr int kDiagSmem = (2 * kNB * kLd + 3 * 32 * 33) * 4;
+constexpr int kDiagSmem = (2 * kNB * kLd + 32 * 100) * 4;
 }  // namespace la
 
 #define GPTQ_TRY(x)               \
@@ -185,196 +185,239 @@ reverse_to_upper_kernel(float* R, const float* Vb, const float* Vs, int64_t n) {
 
 // ------------------------------------------------------------------------------------------------
 // S3/S5 diagonal block: Cholesky of A[k0:k0+nb, k0:k0+nb] on chip (lower; the block's strict upper
-// part is zeroed in A) and the tf32 split of its triangular inverse into (Db, Ds) with ld ldd.
-// Blocked by 32: warp 0 factors each 32 x 32 diagonal piece with its rows in registers (the pivot
-// column is shared through shared memory, pivots use rsqrt and their reciprocals are kept), then
-// inverts the piece while warps 1-3 solve the rows below it by forward substitution; all warps
-// update the trailing part. The off-diagonal pieces of the inverse follow from
-// X[bi][bj] = -X[bi][bi] * sum_k L[bi][k] X[k][bj]. A pivot that is not positive records
-// info_base + k0 + j + 1 (or, for a factorization of the order-reversed matrix of order rev_n > 0,
-// the 1-based index of that pivot in the original order, rev_n - k0 - j) and is replaced by 1 so
-// the remaining arithmetic stays finite.
+// part is zeroed in A when store_l is set) and the tf32 split of its triangular inverse into
+// (Db, Ds) with ld ldd. Blocked by 32-column pieces; for each piece kb:
+//  F  warp 0 factors the piece with its rows in registers and builds the piece's inverse in the
+//     same loop (lane t owns column t of the inverse: X[j][t] = (delta_jt - sum_{m<j} L[j][m]
+//     X[m][t]) / L[j][j], the sums accumulated as the columns of L appear). The pivot of the next
+//     column is updated and broadcast first, so the rest of each column step hides its latency.
+//     Meanwhile warps 1-15 form row block kb-1 of the block's inverse:
+//     X[b][j] = -X[b][b] * sum_m L[b][m] X[m][j] over the pieces already inverted.
+//  S  rows below the piece: L21 = A21 X_kk^T, 4 x 4 register tiles, written transposed into PT;
+//  T  trailing update A22 -= L21 L21^T on lower 4 x 4 tiles read from PT as float4, while PT is
+//     copied back into the panel columns of L.
+// A pivot that is not positive records info_base + k0 + j + 1 (or, for a factorization of the
+// order-reversed matrix of order rev_n > 0, the 1-based index of that pivot in the original
+// order, rev_n - k0 - j) and is replaced by 1 so the remaining arithmetic stays finite.
 // ------------------------------------------------------------------------------------------------
+namespace la {
+constexpr int kLdt = 100;      // PT row: 96 panel rows + pad, a multiple of 4 for float4 access
+}
+
+// Row block b (rows 32b .. 32b+31) of the block's inverse from the pieces already inverted.
+// `part` threads starting at thread `first` take part; `bar` is the barrier between the two
+// products (a named barrier for a subset, or the block barrier).
+__device__ __forceinline__ void diag_inverse_row(const float* L, float* X, float* OT, int b,
+                                                 int part, int first, int bar) {
+  constexpr int LD = la::kLd, LDT = la::kLdt;
+  const int t = threadIdx.x - first;
+  const int items = 64 * b;                       // 8 row groups x 8b column groups of 4 x 4
+  const int rg = t & 7, jg = t >> 3;
+  const int r0 = 32 * b + 4 * rg;
+  if (t < items) {
+    float acc[4][4] = {};
+    for (int m = 32 * (jg >> 3); m < 32 * b; ++m) {
+      float lv[4], xv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) lv[u] = L[(r0 + u) * LD + m];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) xv[v] = X[m * LD + 4 * jg + v];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(lv[u], xv[v], acc[u][v]);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<float4*>(OT + (4 * rg + u) * LDT + 4 * jg) =
+          make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+  }
+  if (bar) named_barrier_or(1, part, false);
+  else __syncthreads();
+  if (t < items) {
+    float acc[4][4] = {};
+    for (int m = 0; m < 4 * rg + 4; ++m) {       // X[b][b] is lower triangular
+      float xb[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) xb[u] = X[(r0 + u) * LD + 32 * b + m];
+      const float4 o = *reinterpret_cast<const float4*>(OT + m * LDT + 4 * jg);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[u][0] = fmaf(xb[u], o.x, acc[u][0]);
+        acc[u][1] = fmaf(xb[u], o.y, acc[u][1]);
+        acc[u][2] = fmaf(xb[u], o.z, acc[u][2]);
+        acc[u][3] = fmaf(xb[u], o.w, acc[u][3]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) X[(r0 + u) * LD + 4 * jg + v] = -acc[u][v];
+  }
+}
+
 __global__ void __launch_bounds__(la::kDiagThreads)
 potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, int64_t ldd,
-                  int32_t* info, int info_base, int rev_n) {
-  constexpr int NB = 128, LD = 129;
+                  int32_t* info, int info_base, int rev_n, int store_l) {
+  constexpr int NB = 128, LD = la::kLd, LDT = la::kLdt;
   extern __shared__ float sm[];
   float* L = sm;
   float* X = sm + NB * LD;
-  float* T = sm + 2 * NB * LD;     // [3][32][33]
-  __shared__ float rdiag[NB];      // 1 / L[j][j]
+  float* PT = sm + 2 * NB * LD;    // [32][LDT]: the panel below the piece, transposed
+  __shared__ float col[64];        // pivot column, double-buffered
   __shared__ int bad;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  constexpr int NW = 16;
   if (tid == 0) bad = -1;
   const bool vec = ((lda & 3) == 0) && ((k0 & 3) == 0) && ((ldd & 3) == 0) &&
                    ((reinterpret_cast<uintptr_t>(A) & 15) == 0) &&
                    ((reinterpret_cast<uintptr_t>(Db) & 15) == 0) &&
                    ((reinterpret_cast<uintptr_t>(Ds) & 15) == 0);
-#pragma unroll 4
-  for (int e = tid; e < NB * NB / 4; e += 512) {
-    const int i = e >> 5, j = (e & 31) * 4;
-    float v[4];
-    if (vec && i < nb && j + 3 < nb) {
-      const float4 q = *reinterpret_cast<const float4*>(A + (k0 + i) * lda + k0 + j);
-      v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
-    } else {
+#pragma unroll 1
+  for (int half = 0; half < 2; ++half) {
+    float v[4][4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = (i < nb && j + u < nb) ? A[(k0 + i) * lda + k0 + j + u] : (i == j + u ? 1.f : 0.f);
+    for (int it = 0; it < 4; ++it) {
+      const int e = tid + (half * 4 + it) * 512;
+      const int i = e >> 5, j = (e & 31) * 4;
+      if (vec && i < nb && j + 3 < nb) {
+        const float4 q = *reinterpret_cast<const float4*>(A + (k0 + i) * lda + k0 + j);
+        v[it][0] = q.x; v[it][1] = q.y; v[it][2] = q.z; v[it][3] = q.w;
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          v[it][u] = (i < nb && j + u < nb) ? A[(k0 + i) * lda + k0 + j + u]
+                                            : (i == j + u ? 1.f : 0.f);
+      }
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) L[i * LD + j + u] = (j + u <= i) ? v[u] : 0.f;
+    for (int it = 0; it < 4; ++it) {
+      const int e = tid + (half * 4 + it) * 512;
+      const int i = e >> 5, j = (e & 31) * 4;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) L[i * LD + j + u] = (j + u <= i) ? v[it][u] : 0.f;
+    }
   }
   __syncthreads();
   for (int kb = 0; kb < 4; ++kb) {
     const int c0 = kb * 32;
     if (warp == 0) {
-      // lane l owns row c0 + l of the 32 x 32 piece, in registers; the pivot column goes through
-      // shared memory (double-buffered, one warp sync per pivot) so each step reads it with
-      // broadcast loads; pivot reciprocals stay in registers until the piece is done
-      float d[32];
+      // ---- F: factor and invert the piece ----
+      // Lane l keeps one register per column k: L[l][k] for k < l (the factor's row) and the
+      // running sum for X[k][l] for k > l (the inverse's column); the diagonal pair L[l][l],
+      // X[l][l] sits in two scalars. Both kinds of entry receive a multiple of the same column
+      // value L[k][j] at step j, so one FMA per register serves both.
+      float e[32];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) d[k] = L[(c0 + lane) * LD + c0 + k];
-      float* col = T;  // 2 x 32-float scratch
-      float rr = 0.f;
+      for (int k = 0; k < 32; ++k) e[k] = (k <= lane) ? L[(c0 + lane) * LD + c0 + k] : 0.f;
+      float ldiag = 1.f, xdiag = 1.f;
       int badj = 32;
-#pragma unroll 32
+      float piv = __shfl_sync(0xffffffffu, e[0], 0);
+#pragma unroll
       for (int j = 0; j < 32; ++j) {
-        const float piv = __shfl_sync(0xffffffffu, d[j], j);
         const bool ok = piv > 0.f && piv < INFINITY;
         const float r = ok ? rsqrtf(piv) : 1.f;
         badj = (!ok && badj == 32) ? j : badj;
-        rr = (lane == j) ? r : rr;
-        const float a = (lane == j) ? (ok ? piv * r : 1.f) : (lane > j ? d[j] * r : 0.f);
-        d[j] = a;
-        col[(j & 1) * 32 + lane] = a;
+        float a, xj;                       // L[l][j] and X[j][l] of this lane
+        if (lane == j) {
+          a = ok ? piv * r : 1.f;
+          xj = r;
+          ldiag = a;
+          xdiag = r;
+        } else if (lane > j) {
+          a = e[j] * r;
+          xj = 0.f;
+          e[j] = a;
+        } else {
+          a = 0.f;
+          xj = -e[j] * r;
+          e[j] = xj;
+        }
+        float* cj = col + (j & 1) * 32;
+        cj[lane] = a;
         __syncwarp();
-#pragma unroll 32
-        for (int k = 0; k < 32; ++k)
-          if (k > j && lane >= k) d[k] = fmaf(-a, col[(j & 1) * 32 + k], d[k]);
+        if (j + 1 < 32) {
+          const float c1 = cj[j + 1];
+          e[j + 1] = fmaf(c1, (lane >= j + 1) ? -a : xj, e[j + 1]);
+          piv = __shfl_sync(0xffffffffu, e[j + 1], j + 1);
+        }
+#pragma unroll
+        for (int k = j + 2; k < 32; ++k) e[k] = fmaf(cj[k], (lane >= k) ? -a : xj, e[k]);
       }
-      rdiag[c0 + lane] = rr;
       if (lane == 0 && badj < 32 && bad < 0) bad = c0 + badj;
 #pragma unroll
-      for (int k = 0; k < 32; ++k) L[(c0 + lane) * LD + c0 + k] = (k <= lane) ? d[k] : 0.f;
+      for (int k = 0; k < 32; ++k) {
+        L[(c0 + lane) * LD + c0 + k] = (k < lane) ? e[k] : (k == lane ? ldiag : 0.f);
+        X[(c0 + k) * LD + c0 + lane] = (k > lane) ? e[k] : (k == lane ? xdiag : 0.f);
+      }
+    } else if (kb >= 2) {
+      // ---- row block kb-1 of the inverse, alongside F ----
+      diag_inverse_row(L, X, PT, kb - 1, NB * 4 - 32, 32, 1);
     }
     __syncthreads();
-    if (warp == 0) {
-      // inverse of the piece: lane t computes column t
-      float x[32];
-#pragma unroll 32
-      for (int i = 0; i < 32; ++i) {
-        float s0 = 0.f, s1 = 0.f;
-#pragma unroll 32
-        for (int m = 0; m < 32; m += 2) {
-          if (m < i && m >= lane) s0 = fmaf(L[(c0 + i) * LD + c0 + m], x[m], s0);
-          if (m + 1 < i && m + 1 >= lane) s1 = fmaf(L[(c0 + i) * LD + c0 + m + 1], x[m + 1], s1);
-        }
-        x[i] = (i < lane) ? 0.f : (((i == lane) ? 1.f : 0.f) - (s0 + s1)) * rdiag[c0 + i];
-      }
-#pragma unroll
-      for (int i = 0; i < 32; ++i) X[(c0 + i) * LD + c0 + lane] = x[i];
-    } else if (c0 + 32 + (warp - 1) * 32 < NB) {
-      // panel below the piece: x P^T = a by forward substitution, lane = row
-      const int r = c0 + 32 + (warp - 1) * 32 + lane;
-      float x[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) x[c] = L[r * LD + c0 + c];
-#pragma unroll 32
-      for (int c = 0; c < 32; ++c) {
-        float s0 = x[c], s1 = 0.f;
-#pragma unroll 32
-        for (int m = 0; m < 32; m += 2) {
-          if (m < c) s0 = fmaf(-x[m], L[(c0 + c) * LD + c0 + m], s0);
-          if (m + 1 < c) s1 = fmaf(-x[m + 1], L[(c0 + c) * LD + c0 + m + 1], s1);
-        }
-        x[c] = (s0 + s1) * rdiag[c0 + c];
-      }
-#pragma unroll
-      for (int c = 0; c < 32; ++c) L[r * LD + c0 + c] = x[c];
-    }
-    __syncthreads();
-    // trailing update: lane owns column l (panel values in registers); rows i >= l in steps of 4,
-    // two rows at a time
+    const int nbelow = NB - c0 - 32;
+    if (nbelow == 0) break;
+    // ---- S: L21 = A21 X_kk^T into PT (transposed) ----
     {
-      const int base = c0 + 32;
-      const int ncol = NB - base;
-      for (int t = warp * 32; t < ncol * 4; t += NW * 32) {
-        const int item = t + lane;
-        if (item < ncol * 4) {
-          const int l = base + item % ncol;
-          const int g = item / ncol;
-          float pv[32];
+      const int nrq = nbelow / 4;
+      if (tid < nrq * 8) {
+        const int cg = (tid >> 3) & 7, rq = (tid & 7) + 8 * (tid >> 6);
+        const int rr = c0 + 32 + 4 * rq;
+        float acc[4][4] = {};
+        for (int m = 0; m < 4 * cg + 4; ++m) {   // X_kk[c][m] = 0 for m > c
+          float av[4], xv[4];
 #pragma unroll
-          for (int m = 0; m < 32; ++m) pv[m] = L[l * LD + c0 + m];
-          int i = l + g;
-          for (; i + 4 < NB; i += 8) {
-            float s0 = 0.f, s1 = 0.f, u0 = 0.f, u1 = 0.f;
+          for (int u = 0; u < 4; ++u) av[u] = L[(rr + u) * LD + c0 + m];
 #pragma unroll
-            for (int m = 0; m < 32; m += 2) {
-              s0 = fmaf(L[i * LD + c0 + m], pv[m], s0);
-              s1 = fmaf(L[i * LD + c0 + m + 1], pv[m + 1], s1);
-              u0 = fmaf(L[(i + 4) * LD + c0 + m], pv[m], u0);
-              u1 = fmaf(L[(i + 4) * LD + c0 + m + 1], pv[m + 1], u1);
-            }
-            L[i * LD + l] -= s0 + s1;
-            L[(i + 4) * LD + l] -= u0 + u1;
-          }
-          if (i < NB) {
-            float s0 = 0.f, s1 = 0.f;
+          for (int v = 0; v < 4; ++v) xv[v] = X[(c0 + 4 * cg + v) * LD + c0 + m];
 #pragma unroll
-            for (int m = 0; m < 32; m += 2) {
-              s0 = fmaf(L[i * LD + c0 + m], pv[m], s0);
-              s1 = fmaf(L[i * LD + c0 + m + 1], pv[m + 1], s1);
-            }
-            L[i * LD + l] -= s0 + s1;
-          }
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], xv[v], acc[u][v]);
         }
+#pragma unroll
+        for (int v = 0; v < 4; ++v)
+          *reinterpret_cast<float4*>(PT + (4 * cg + v) * LDT + 4 * rq) =
+              make_float4(acc[0][v], acc[1][v], acc[2][v], acc[3][v]);
+      }
+    }
+    __syncthreads();
+    // ---- T: A22 -= L21 L21^T (lower 4 x 4 tiles), and PT back into L's panel columns ----
+    {
+      const int nb4 = nbelow / 4;
+      const int nblk = nb4 * (nb4 + 1) / 2;
+      for (int blk = tid; blk < nblk; blk += 512) {
+        int bi, bl;
+        decode_tri(blk, bi, bl);
+        float acc[4][4] = {};
+#pragma unroll 8
+        for (int m = 0; m < 32; ++m) {
+          const float4 a4 = *reinterpret_cast<const float4*>(PT + m * LDT + 4 * bi);
+          const float4 b4 = *reinterpret_cast<const float4*>(PT + m * LDT + 4 * bl);
+          const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+        }
+        const int i0 = c0 + 32 + 4 * bi, l0 = c0 + 32 + 4 * bl;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            if (l0 + v <= i0 + u) L[(i0 + u) * LD + l0 + v] -= acc[u][v];
+      }
+      for (int e = tid; e < nbelow * 32; e += 512) {
+        const int r = e >> 5, c = e & 31;
+        L[(c0 + 32 + r) * LD + c0 + c] = PT[c * LDT + r];
       }
     }
     __syncthreads();
   }
   if (tid == 0 && bad >= 0 && bad < nb)
     record_info(info, rev_n > 0 ? rev_n - (k0 + bad) : info_base + k0 + bad + 1);
-  // off-diagonal pieces of the inverse, 2 x 2 outputs per thread (rows r, r+16; cols c, c+16)
-  for (int bi = 1; bi < 4; ++bi) {
-    for (int e = tid; e < bi * 256; e += 512) {
-      const int bj = e >> 8, r = (e >> 4) & 15, c = e & 15;
-      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
-      const float* l0 = L + (32 * bi + r) * LD;
-      const float* l1 = L + (32 * bi + r + 16) * LD;
-      for (int k = 32 * bj; k < 32 * bi; ++k) {
-        const float x0 = X[k * LD + 32 * bj + c], x1 = X[k * LD + 32 * bj + c + 16];
-        const float p0 = l0[k], p1 = l1[k];
-        a00 = fmaf(p0, x0, a00); a01 = fmaf(p0, x1, a01);
-        a10 = fmaf(p1, x0, a10); a11 = fmaf(p1, x1, a11);
-      }
-      float* t = T + bj * 32 * 33;
-      t[r * 33 + c] = a00; t[r * 33 + c + 16] = a01;
-      t[(r + 16) * 33 + c] = a10; t[(r + 16) * 33 + c + 16] = a11;
-    }
-    __syncthreads();
-    for (int e = tid; e < bi * 256; e += 512) {
-      const int bj = e >> 8, r = (e >> 4) & 15, c = e & 15;
-      float a00 = 0.f, a01 = 0.f, a10 = 0.f, a11 = 0.f;
-      const float* x0r = X + (32 * bi + r) * LD + 32 * bi;
-      const float* x1r = X + (32 * bi + r + 16) * LD + 32 * bi;
-      const float* t = T + bj * 32 * 33;
-#pragma unroll 8
-      for (int m = 0; m < 32; ++m) {
-        const float t0 = t[m * 33 + c], t1 = t[m * 33 + c + 16];
-        const float p0 = x0r[m], p1 = x1r[m];
-        a00 = fmaf(p0, t0, a00); a01 = fmaf(p0, t1, a01);
-        a10 = fmaf(p1, t0, a10); a11 = fmaf(p1, t1, a11);
-      }
-      float* xo = X + (32 * bi) * LD + 32 * bj;
-      xo[r * LD + c] = -a00; xo[r * LD + c + 16] = -a01;
-      xo[(r + 16) * LD + c] = -a10; xo[(r + 16) * LD + c + 16] = -a11;
-    }
-    __syncthreads();
-  }
+  // the last row block of the inverse, with every thread
+  diag_inverse_row(L, X, PT, 3, NB * 4, 0, 0);
+  __syncthreads();
 #pragma unroll 4
   for (int e = tid; e < NB * NB / 4; e += 512) {
     const int i = e >> 5, j = (e & 31) * 4;
@@ -389,14 +432,16 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
       sv[u] = x - bv[u];
     }
     if (vec && j + 3 < nb) {
-      *reinterpret_cast<float4*>(A + (k0 + i) * lda + k0 + j) = make_float4(lv[0], lv[1], lv[2], lv[3]);
+      if (store_l)
+        *reinterpret_cast<float4*>(A + (k0 + i) * lda + k0 + j) =
+            make_float4(lv[0], lv[1], lv[2], lv[3]);
       *reinterpret_cast<float4*>(Db + i * ldd + j) = make_float4(bv[0], bv[1], bv[2], bv[3]);
       *reinterpret_cast<float4*>(Ds + i * ldd + j) = make_float4(sv[0], sv[1], sv[2], sv[3]);
     } else {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         if (j + u >= nb) continue;
-        A[(k0 + i) * lda + k0 + j + u] = lv[u];
+        if (store_l) A[(k0 + i) * lda + k0 + j + u] = lv[u];
         Db[i * ldd + j + u] = bv[u];
         Ds[i * ldd + j + u] = sv[u];
       }
@@ -406,7 +451,7 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
 
 static gptq_status launch_potrf_diag(float* A, int64_t n, int k0, int nb, float* Db, float* Ds,
                                      int64_t ldd, int32_t* info, int info_base, int rev_n,
-                                     cudaStream_t stream) {
+                                     bool store_l, cudaStream_t stream) {
   static bool attr_done = false;
   if (!attr_done) {
     if (cudaFuncSetAttribute(potrf_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -415,7 +460,7 @@ static gptq_status launch_potrf_diag(float* A, int64_t n, int k0, int nb, float*
     attr_done = true;
   }
   potrf_diag_kernel<<<1, la::kDiagThreads, la::kDiagSmem, stream>>>(A, n, k0, nb, Db, Ds, ldd, info,
-                                                                     info_base, rev_n);
+                                                                     info_base, rev_n, store_l);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }
@@ -430,16 +475,18 @@ struct Split {
 //   Dsp:  where each diagonal block's inverse goes (ld ld_dinv): at block k0 of an n x n matrix
 //         when per_block is set (the block diagonal of L^-1), else one shared 128 x 128 scratch;
 //   Psp:  split of the current panel before its solve (n x 128);
-//   rev_n: > 0 when A is the order-reversed matrix (pivot codes then name original columns).
+//   rev_n: > 0 when A is the order-reversed matrix (pivot codes then name original columns);
+//   store_l: write the factored diagonal blocks back into A (only needed when A's own lower
+//         triangle is the result; the panels below them are always written).
 static gptq_status potrf_blocked(float* A, int64_t n, Split Lsp, Split Dsp, int64_t ld_dinv,
                                  bool per_block, Split Psp, int32_t* info, int info_base,
-                                 int rev_n, cudaStream_t stream) {
+                                 int rev_n, bool store_l, cudaStream_t stream) {
   using namespace la;
   for (int64_t k0 = 0; k0 < n; k0 += kNB) {
     const int nb = static_cast<int>(n - k0 < kNB ? n - k0 : kNB);
     const int64_t doff = per_block ? k0 * ld_dinv + k0 : 0;
     GPTQ_TRY(launch_potrf_diag(A, n, static_cast<int>(k0), nb, Dsp.b + doff, Dsp.s + doff, ld_dinv,
-                               info, info_base, rev_n, stream));
+                               info, info_base, rev_n, store_l, stream));
     const int64_t m = n - k0 - nb;
     if (m == 0) break;
     float* A21 = A + (k0 + nb) * n + k0;
@@ -554,7 +601,7 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
   // S3: H_d = L L^T in R (reversed route: J H_d J = M M^T, M written as L below); the inverses of
   // L's diagonal blocks land in V (the split of L^-1)
   GPTQ_TRY(potrf_blocked(R, n, w.L, w.V, n, true, w.P, info, 0, reversed ? static_cast<int>(n) : 0,
-                         stream));
+                         false, stream));
 
   // S4a: the rest of L^-1 by recursive doubling over the diagonal blocks already inverted.
   GPTQ_TRY(trtri_doubling(w, n, info, stream));
@@ -573,7 +620,8 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
   GPTQ_TRY(launch_gemm_tc(h, stream));
 
   // S5: H_d^-1 = L2 L2^T (reusing the L split and the diagonal scratch), then R = L2^T
-  GPTQ_TRY(potrf_blocked(R, n, w.L, w.D, kNB, false, w.P, info, static_cast<int>(n), 0, stream));
+  GPTQ_TRY(potrf_blocked(R, n, w.L, w.D, kNB, false, w.P, info, static_cast<int>(n), 0, true,
+                         stream));
   transpose_to_upper_kernel<<<ntri, dim3(32, 8), 0, stream>>>(R, n);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
