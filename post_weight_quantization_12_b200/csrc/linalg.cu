@@ -15,6 +15,7 @@
 // Each 128 x 128 diagonal block is factored and inverted on chip by one CTA; everything else is a
 // 3xTF32 tensor-core matrix product whose operands are kept as tf32 (big, small) pairs in the
 // workspace.
+#include <climits>
 #include <cmath>
 
 #include "common.cuh"
@@ -26,7 +27,7 @@ namespace la {
 constexpr int kNB = 128;       // panel / diagonal block width
 constexpr int kLd = kNB + 1;   // padded shared-memory row
 constexpr int kDiagThreads = 512;
-constexpr int kDiagSmem = (2 * kNB * kLd + 32 * 100) * 4;
+constexpr int kDiagSmem = (2 * kNB * kLd + 3 * 32 * 100) * 4;
 }  // namespace la
 
 #define GPTQ_TRY(x)               \
@@ -187,12 +188,15 @@ reverse_to_upper_kernel(float* R, const float* Vb, const float* Vs, int64_t n) {
 // S3/S5 diagonal block: Cholesky of A[k0:k0+nb, k0:k0+nb] on chip (lower; the block's strict upper
 // part is zeroed in A when store_l is set) and the tf32 split of its triangular inverse into
 // (Db, Ds) with ld ldd. Blocked by 32-column pieces; for each piece kb:
-//  F  warp 0 factors the piece with its rows in registers and builds the piece's inverse in the
-//     same loop (lane t owns column t of the inverse: X[j][t] = (delta_jt - sum_{m<j} L[j][m]
-//     X[m][t]) / L[j][j], the sums accumulated as the columns of L appear). The pivot of the next
-//     column is updated and broadcast first, so the rest of each column step hides its latency.
-//     Meanwhile warps 1-15 form row block kb-1 of the block's inverse:
-//     X[b][j] = -X[b][b] * sum_m L[b][m] X[m][j] over the pieces already inverted.
+//  F  warp 0 factors the piece and builds its inverse in the same loop. Lane l is row l and keeps
+//     one register per column k: L[l][k] for k < l (the factor's row) or the running sum for
+//     X[k][l] for k > l (the inverse's column, X[j][t] = (delta_jt - sum_{m<j} L[j][m] X[m][t]) /
+//     L[j][j]); the diagonal pair L[l][l], X[l][l] sits in two scalars. Both kinds of entry
+//     receive a multiple of the same column value L[k][j] at step j, so one FMA per register
+//     serves both. The next pivot is updated and broadcast before the rest of each column step.
+//     Meanwhile warps 1-15 form the block's inverse row blocks,
+//     X[b][j] = -X[b][b] * sum_m L[b][m] X[m][j]: the sum for row block kb and the product with
+//     X[kb-1][kb-1] for row block kb-1.
 //  S  rows below the piece: L21 = A21 X_kk^T, 4 x 4 register tiles, written transposed into PT;
 //  T  trailing update A22 -= L21 L21^T on lower 4 x 4 tiles read from PT as float4, while PT is
 //     copied back into the panel columns of L.
@@ -201,59 +205,63 @@ reverse_to_upper_kernel(float* R, const float* Vb, const float* Vs, int64_t n) {
 // order, rev_n - k0 - j) and is replaced by 1 so the remaining arithmetic stays finite.
 // ------------------------------------------------------------------------------------------------
 namespace la {
-constexpr int kLdt = 100;      // PT row: 96 panel rows + pad, a multiple of 4 for float4 access
+constexpr int kLdt = 100;      // PT / OT row: 96 entries + pad, a multiple of 4 for float4 access
+constexpr int kInverseBar = 1;
+constexpr int kInverseThreads = kDiagThreads - 32;
 }
 
-// Row block b (rows 32b .. 32b+31) of the block's inverse from the pieces already inverted.
-// `part` threads starting at thread `first` take part; `bar` is the barrier between the two
-// products (a named barrier for a subset, or the block barrier).
-__device__ __forceinline__ void diag_inverse_row(const float* L, float* X, float* OT, int b,
-                                                 int part, int first, int bar) {
+// First half of row block b of the inverse: OT[r][j] = sum_m L[32b + r][m] X[m][j], j < 32b, over
+// the row blocks already inverted. Threads first .. first + 64b - 1 take part (4 x 4 tiles).
+__device__ __forceinline__ void inverse_row_sum(const float* L, const float* X, float* OT, int b,
+                                                int first) {
   constexpr int LD = la::kLd, LDT = la::kLdt;
   const int t = threadIdx.x - first;
-  const int items = 64 * b;                       // 8 row groups x 8b column groups of 4 x 4
+  if (t < 0 || t >= 64 * b) return;
   const int rg = t & 7, jg = t >> 3;
   const int r0 = 32 * b + 4 * rg;
-  if (t < items) {
-    float acc[4][4] = {};
-    for (int m = 32 * (jg >> 3); m < 32 * b; ++m) {
-      float lv[4], xv[4];
+  float acc[4][4] = {};
+  for (int m = 32 * (jg >> 3); m < 32 * b; ++m) {
+    float lv[4], xv[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) lv[u] = L[(r0 + u) * LD + m];
+    for (int u = 0; u < 4; ++u) lv[u] = L[(r0 + u) * LD + m];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) xv[v] = X[m * LD + 4 * jg + v];
-#pragma unroll
-      for (int u = 0; u < 4; ++u)
-#pragma unroll
-        for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(lv[u], xv[v], acc[u][v]);
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u)
-      *reinterpret_cast<float4*>(OT + (4 * rg + u) * LDT + 4 * jg) =
-          make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
-  }
-  if (bar) named_barrier_or(1, part, false);
-  else __syncthreads();
-  if (t < items) {
-    float acc[4][4] = {};
-    for (int m = 0; m < 4 * rg + 4; ++m) {       // X[b][b] is lower triangular
-      float xb[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) xb[u] = X[(r0 + u) * LD + 32 * b + m];
-      const float4 o = *reinterpret_cast<const float4*>(OT + m * LDT + 4 * jg);
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc[u][0] = fmaf(xb[u], o.x, acc[u][0]);
-        acc[u][1] = fmaf(xb[u], o.y, acc[u][1]);
-        acc[u][2] = fmaf(xb[u], o.z, acc[u][2]);
-        acc[u][3] = fmaf(xb[u], o.w, acc[u][3]);
-      }
-    }
+    for (int v = 0; v < 4; ++v) xv[v] = X[m * LD + 4 * jg + v];
 #pragma unroll
     for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int v = 0; v < 4; ++v) X[(r0 + u) * LD + 4 * jg + v] = -acc[u][v];
+      for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(lv[u], xv[v], acc[u][v]);
   }
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    *reinterpret_cast<float4*>(OT + (4 * rg + u) * LDT + 4 * jg) =
+        make_float4(acc[u][0], acc[u][1], acc[u][2], acc[u][3]);
+}
+
+// Second half: X[32b + r][j] = -sum_{m <= r} X[32b + r][32b + m] OT[m][j].
+__device__ __forceinline__ void inverse_row_product(float* X, const float* OT, int b, int first) {
+  constexpr int LD = la::kLd, LDT = la::kLdt;
+  const int t = threadIdx.x - first;
+  if (t < 0 || t >= 64 * b) return;
+  const int rg = t & 7, jg = t >> 3;
+  const int r0 = 32 * b + 4 * rg;
+  float acc[4][4] = {};
+  for (int m = 0; m < 4 * rg + 4; ++m) {         // X[b][b] is lower triangular
+    float xb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) xb[u] = X[(r0 + u) * LD + 32 * b + m];
+    const float4 o = *reinterpret_cast<const float4*>(OT + m * LDT + 4 * jg);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      acc[u][0] = fmaf(xb[u], o.x, acc[u][0]);
+      acc[u][1] = fmaf(xb[u], o.y, acc[u][1]);
+      acc[u][2] = fmaf(xb[u], o.z, acc[u][2]);
+      acc[u][3] = fmaf(xb[u], o.w, acc[u][3]);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v) X[(r0 + u) * LD + 4 * jg + v] = -acc[u][v];
 }
 
 __global__ void __launch_bounds__(la::kDiagThreads)
@@ -264,14 +272,16 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
   float* L = sm;
   float* X = sm + NB * LD;
   float* PT = sm + 2 * NB * LD;    // [32][LDT]: the panel below the piece, transposed
+  float* OT = PT + 32 * LDT;       // 2 x [32][LDT]: partial sums of inverse row blocks
   __shared__ float col[64];        // pivot column, double-buffered
-  __shared__ int bad;
+  __shared__ int bad;              // first pivot that was not positive (INT_MAX: none)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) bad = -1;
+  if (tid == 0) bad = INT_MAX;
   const bool vec = ((lda & 3) == 0) && ((k0 & 3) == 0) && ((ldd & 3) == 0) &&
                    ((reinterpret_cast<uintptr_t>(A) & 15) == 0) &&
                    ((reinterpret_cast<uintptr_t>(Db) & 15) == 0) &&
                    ((reinterpret_cast<uintptr_t>(Ds) & 15) == 0);
+  // load the block (outside nb: identity)
 #pragma unroll 1
   for (int half = 0; half < 2; ++half) {
     float v[4][4];
@@ -298,14 +308,11 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
     }
   }
   __syncthreads();
+#pragma unroll 1
   for (int kb = 0; kb < 4; ++kb) {
     const int c0 = kb * 32;
     if (warp == 0) {
       // ---- F: factor and invert the piece ----
-      // Lane l keeps one register per column k: L[l][k] for k < l (the factor's row) and the
-      // running sum for X[k][l] for k > l (the inverse's column); the diagonal pair L[l][l],
-      // X[l][l] sits in two scalars. Both kinds of entry receive a multiple of the same column
-      // value L[k][j] at step j, so one FMA per register serves both.
       float e[32];
 #pragma unroll
       for (int k = 0; k < 32; ++k) e[k] = (k <= lane) ? L[(c0 + lane) * LD + c0 + k] : 0.f;
@@ -343,15 +350,20 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
 #pragma unroll
         for (int k = j + 2; k < 32; ++k) e[k] = fmaf(cj[k], (lane >= k) ? -a : xj, e[k]);
       }
-      if (lane == 0 && badj < 32 && bad < 0) bad = c0 + badj;
+      if (lane == 0 && badj < 32) atomicMin(&bad, c0 + badj);
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
         L[(c0 + lane) * LD + c0 + k] = (k < lane) ? e[k] : (k == lane ? ldiag : 0.f);
         X[(c0 + k) * LD + c0 + lane] = (k > lane) ? e[k] : (k == lane ? xdiag : 0.f);
       }
-    } else if (kb >= 2) {
-      // ---- row block kb-1 of the inverse, alongside F ----
-      diag_inverse_row(L, X, PT, kb - 1, NB * 4 - 32, 32, 1);
+    } else {
+      // ---- inverse row blocks, alongside F (warps 1-15) ----
+      const int first = 32;
+      if (kb >= 2) {
+        inverse_row_product(X, OT + ((kb - 1) & 1) * 32 * LDT, kb - 1, first);
+        named_barrier_or(la::kInverseBar, la::kInverseThreads, false);
+      }
+      if (kb >= 1) inverse_row_sum(L, X, OT + (kb & 1) * 32 * LDT, kb, first);
     }
     __syncthreads();
     const int nbelow = NB - c0 - 32;
@@ -413,11 +425,12 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
     }
     __syncthreads();
   }
-  if (tid == 0 && bad >= 0 && bad < nb)
+  if (tid == 0 && bad < nb)
     record_info(info, rev_n > 0 ? rev_n - (k0 + bad) : info_base + k0 + bad + 1);
-  // the last row block of the inverse, with every thread
-  diag_inverse_row(L, X, PT, 3, NB * 4, 0, 0);
+  // the last row block of the inverse (its sums were formed alongside the last piece)
+  inverse_row_product(X, OT + 1 * 32 * LDT, 3, 0);
   __syncthreads();
+  // store: L when asked, and the tf32 split of the inverse
 #pragma unroll 4
   for (int e = tid; e < NB * NB / 4; e += 512) {
     const int i = e >> 5, j = (e & 31) * 4;
