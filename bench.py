@@ -39,8 +39,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # Nominal dense tf32 / bf16 throughput ratio (1.1 / 2.25 PFLOP/s); tf32 has no measured peak here.
 TF32_PER_BF16 = 1.1 / 2.25
 # DRAM traffic of the S1 kernel from one ncu capture of 16384 tokens x 4096 channels (reads scale
-# with tokens -- X is streamed once per round of tiles; writes are S, once per launch).
-SYRK_CAPTURE = {"tokens": 16384, "cols": 4096, "dram_read": 269.261e6, "dram_write": 26.181e6}
+# with tokens -- X is streamed once per round of tiles; writes are S, once per launch). None until
+# the current kernel has been captured.
+SYRK_CAPTURE = None
 
 
 def parse():
@@ -346,7 +347,7 @@ def run_ours(args):
     achieved = flops / t_syrk / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     traffic = None
-    if cols == SYRK_CAPTURE["cols"]:
+    if SYRK_CAPTURE and cols == SYRK_CAPTURE["cols"]:
         traffic = SYRK_CAPTURE["dram_read"] * n / SYRK_CAPTURE["tokens"] + SYRK_CAPTURE["dram_write"]
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                 "frac": achieved / peak, "traffic": traffic,

@@ -6,12 +6,14 @@
 // bf16 path: a persistent tcgen05 SYRK on CTA pairs (the 2-SM form, cta_group::2). The output is
 // cut into 256 x 256 lower-triangle super-tiles; each pair of CTAs (a cluster of 2 on two SMs) owns
 // one super-tile per round and walks the whole token range for it, so all pairs read the same token
-// slab at about the same time (fetched from HBM once, served to the others from L2). Per 32-token
+// slab at about the same time (fetched from HBM once, served to the others from L2). Per 128-token
 // stage each CTA brings, by TMA with 128-byte swizzle, the 128 channels of its half of the rows (A)
-// and of its half of the columns (B) into its own shared memory (16 KB); both operands are MN-major
-// (channels contiguous), which tcgen05 reads directly, and on a diagonal super-tile A doubles as B.
-// The first CTA of the pair issues two 256 x 256 x 16 MMAs per stage; each CTA's TMEM receives its
-// 128 rows. Per SM this moves half the operand bytes of a 128 x 256 single-SM tile.
+// and of its half of the columns (B) into its own shared memory (64 KB, three stages); both
+// operands are MN-major (channels contiguous), which tcgen05 reads directly, and on a diagonal
+// super-tile A doubles as B. The first CTA of the pair issues eight 256 x 256 x 16 MMAs per stage;
+// each CTA's TMEM receives its 128 rows. Per SM this moves half the operand bytes of a 128 x 256
+// single-SM tile. Long stages matter: with 32-token stages (4 KB boxes) the same pipeline kept the
+// tensor cores waiting for operands a third of the time.
 //
 // The tensor core adds each MMA's products into its fp32 accumulator with a rounding biased
 // toward zero, so the relative error of one TMEM sum grows with the number of MMAs folded into it
@@ -28,16 +30,16 @@
 namespace gptq {
 
 namespace syrk {
-constexpr int kBK = 32;                    // tokens per stage
-constexpr int kStages = 12;
+constexpr int kBK = 128;                   // tokens per stage
+constexpr int kStages = 3;
 constexpr int kBoxCh = 64;                 // channels per TMA box (128 bytes of bf16)
-constexpr int kBoxBytes = kBoxCh * kBK * 2;          // 4 KB
+constexpr int kBoxBytes = kBoxCh * kBK * 2;          // 16 KB
 constexpr int kHalfBytes = 2 * kBoxBytes;            // 128 channels
-constexpr int kStageBytes = 2 * kHalfBytes;          // A half + B half: 16 KB per CTA
+constexpr int kStageBytes = 2 * kHalfBytes;          // A half + B half: 64 KB per CTA
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;
 constexpr int kThreads = 320;              // warp 0 TMA, warp 1 MMA (first CTA), warps 2-9 fold
 constexpr uint32_t kTmemCols = 512;        // two 256-column chunk accumulators (128 rows each)
-constexpr int kChunkStages = 64;           // 2048 tokens per TMEM chunk sum
+constexpr int kChunkStages = 2048 / kBK;   // 2048 tokens per TMEM chunk sum
 constexpr uint32_t kIdesc = make_idesc(/*bf16*/ 1, /*A MN-major*/ 1, /*B MN-major*/ 1, 256, 256);
 constexpr int kEpiWarps = 8;
 }  // namespace syrk
