@@ -188,12 +188,8 @@ reverse_to_upper_kernel(float* R, const float* Vb, const float* Vs, int64_t n) {
 // S3/S5 diagonal block: Cholesky of A[k0:k0+nb, k0:k0+nb] on chip (lower; the block's strict upper
 // part is zeroed in A when store_l is set) and the tf32 split of its triangular inverse into
 // (Db, Ds) with ld ldd. Blocked by 32-column pieces; for each piece kb:
-//  F  warp 0 factors the piece and builds its inverse in the same loop. Lane l is row l and keeps
-//     one register per column k: L[l][k] for k < l (the factor's row) or the running sum for
-//     X[k][l] for k > l (the inverse's column, X[j][t] = (delta_jt - sum_{m<j} L[j][m] X[m][t]) /
-//     L[j][j]); the diagonal pair L[l][l], X[l][l] sits in two scalars. Both kinds of entry
-//     receive a multiple of the same column value L[k][j] at step j, so one FMA per register
-//     serves both. The next pivot is updated and broadcast before the rest of each column step.
+//  F  warp 0 factors the piece and builds its inverse in the same loop, four columns per step
+//     (factor_piece4).
 //     Meanwhile warps 1-15 form the block's inverse row blocks,
 //     X[b][j] = -X[b][b] * sum_m L[b][m] X[m][j]: the sum for row block kb and the product with
 //     X[kb-1][kb-1] for row block kb-1.
@@ -264,6 +260,82 @@ __device__ __forceinline__ void inverse_row_product(float* X, const float* OT, i
     for (int v = 0; v < 4; ++v) X[(r0 + u) * LD + 4 * jg + v] = -acc[u][v];
 }
 
+// Factor and invert one 32 x 32 piece in one warp, four columns per step. Lane l is row l; e[k]
+// holds L[l][k] for k < l (the factor's row) and the running sum for X[k][l] for k > l (the
+// inverse's column, X[j][t] = (delta_jt - sum_{m<j} L[j][m] X[m][t]) / L[j][j]); the diagonal pair
+// L[l][l], X[l][l] ends in ldiag / xdiag. Per step every lane factors the step's 4 x 4 diagonal
+// block itself (broadcast by shuffles), solves its own four entries of L or X, and applies the
+// four new columns to its remaining registers: entries of L take -L[l][j] L[k][j], entries of X
+// take L[k][j] X[j][l], so one FMA per register and column serves both. `col` holds two 32-entry
+// buffers. A pivot that is not positive is replaced by 1 and its index goes to badj.
+__device__ __forceinline__ void factor_piece4(float (&e)[32], float& ldiag, float& xdiag, int& badj,
+                                              float4* col, int lane) {
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const int j = 4 * t;
+    float b[4][4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+      for (int q = 0; q <= p; ++q) b[p][q] = __shfl_sync(0xffffffffu, e[j + q], j + p);
+    float lb[4][4], r[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float d = b[q][q];
+#pragma unroll
+      for (int s = 0; s < q; ++s) d = fmaf(-lb[q][s], lb[q][s], d);
+      const bool ok = d > 0.f && d < INFINITY;
+      r[q] = ok ? rsqrtf(d) : 1.f;
+      lb[q][q] = ok ? d * r[q] : 1.f;
+      badj = (!ok && badj == 32) ? j + q : badj;
+#pragma unroll
+      for (int p = q + 1; p < 4; ++p) {
+        float v = b[p][q];
+#pragma unroll
+        for (int s = 0; s < q; ++s) v = fmaf(-lb[p][s], lb[q][s], v);
+        lb[p][q] = v * r[q];
+      }
+    }
+    float a[4], x[4];                      // L[lane][j+q] and X[j+q][lane]
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int k = j + q;
+      float sa = e[k], sx = -e[k];
+#pragma unroll
+      for (int s = 0; s < q; ++s) {
+        sa = fmaf(-a[s], lb[q][s], sa);
+        sx = fmaf(-lb[q][s], x[s], sx);
+      }
+      if (lane > k) {
+        a[q] = sa * r[q];
+        x[q] = 0.f;
+        e[k] = a[q];
+      } else if (lane == k) {
+        a[q] = lb[q][q];
+        x[q] = r[q];
+        ldiag = lb[q][q];
+        xdiag = r[q];
+      } else {
+        a[q] = 0.f;
+        x[q] = sx * r[q];
+        e[k] = x[q];
+      }
+    }
+    float4* cb = col + (t & 1) * 32;
+    cb[lane] = make_float4(a[0], a[1], a[2], a[3]);
+    __syncwarp();
+#pragma unroll
+    for (int k = j + 4; k < 32; ++k) {
+      const float4 c = cb[k];
+      const bool fac = lane >= k;
+      e[k] = fmaf(c.x, fac ? -a[0] : x[0], e[k]);
+      e[k] = fmaf(c.y, fac ? -a[1] : x[1], e[k]);
+      e[k] = fmaf(c.z, fac ? -a[2] : x[2], e[k]);
+      e[k] = fmaf(c.w, fac ? -a[3] : x[3], e[k]);
+    }
+  }
+}
+
 __global__ void __launch_bounds__(la::kDiagThreads)
 potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, int64_t ldd,
                   int32_t* info, int info_base, int rev_n, int store_l) {
@@ -273,7 +345,7 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
   float* X = sm + NB * LD;
   float* PT = sm + 2 * NB * LD;    // [32][LDT]: the panel below the piece, transposed
   float* OT = PT + 32 * LDT;       // 2 x [32][LDT]: partial sums of inverse row blocks
-  __shared__ float col[64];        // pivot column, double-buffered
+  __shared__ float4 col4[64];     // four new columns per step, double-buffered
   __shared__ int bad;              // first pivot that was not positive (INT_MAX: none)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) bad = INT_MAX;
@@ -318,38 +390,7 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
       for (int k = 0; k < 32; ++k) e[k] = (k <= lane) ? L[(c0 + lane) * LD + c0 + k] : 0.f;
       float ldiag = 1.f, xdiag = 1.f;
       int badj = 32;
-      float piv = __shfl_sync(0xffffffffu, e[0], 0);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const bool ok = piv > 0.f && piv < INFINITY;
-        const float r = ok ? rsqrtf(piv) : 1.f;
-        badj = (!ok && badj == 32) ? j : badj;
-        float a, xj;                       // L[l][j] and X[j][l] of this lane
-        if (lane == j) {
-          a = ok ? piv * r : 1.f;
-          xj = r;
-          ldiag = a;
-          xdiag = r;
-        } else if (lane > j) {
-          a = e[j] * r;
-          xj = 0.f;
-          e[j] = a;
-        } else {
-          a = 0.f;
-          xj = -e[j] * r;
-          e[j] = xj;
-        }
-        float* cj = col + (j & 1) * 32;
-        cj[lane] = a;
-        __syncwarp();
-        if (j + 1 < 32) {
-          const float c1 = cj[j + 1];
-          e[j + 1] = fmaf(c1, (lane >= j + 1) ? -a : xj, e[j + 1]);
-          piv = __shfl_sync(0xffffffffu, e[j + 1], j + 1);
-        }
-#pragma unroll
-        for (int k = j + 2; k < 32; ++k) e[k] = fmaf(cj[k], (lane >= k) ? -a : xj, e[k]);
-      }
+      factor_piece4(e, ldiag, xdiag, badj, col4, lane);
       if (lane == 0 && badj < 32) atomicMin(&bad, c0 + badj);
 #pragma unroll
       for (int k = 0; k < 32; ++k) {
