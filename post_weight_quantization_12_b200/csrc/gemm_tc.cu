@@ -307,7 +307,8 @@ constexpr int kStageBytes = 4 * kPartBytes;         // A_big, A_small, B_big, B_
 constexpr int kBoxBytes = BM * 32 * 4;              // 16 KB: 128 rows x 32 columns of C
 constexpr int kSmemBytes = kStages * kStageBytes + 1024;
 constexpr int kSmemBytesStaged = kSmemBytes + 4 * kBoxBytes;
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;                       // warps: 0 A/B loads, 1 MMA, 2-5 epilogue, 6 C
+constexpr int kIssuerWarp = 6;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kEpiBarrier = 1;                 // named barrier of the 128 epilogue threads
 }  // namespace tgp
@@ -321,7 +322,9 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
-  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done, c_full[4];
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
+  __shared__ __align__(8) uint64_t cbox[4];        // box j may be written (and holds C if beta != 0)
+  __shared__ __align__(8) uint64_t ready[4];       // box j written by the epilogue, may be stored
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
@@ -338,7 +341,10 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], 128);
     }
-    for (int j = 0; j < 4; ++j) mbar_init(&c_full[j], 1);
+    for (int j = 0; j < 4; ++j) {
+      mbar_init(&cbox[j], 1);
+      mbar_init(&ready[j], 128);
+    }
     mbar_init(&mma_done, 1);
     abort_flag = 0;
     fence_mbarrier_init();
@@ -434,42 +440,86 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
       tc_commit(&mma_done);
       mbar_drain_bounded(&mma_done, 0);
     }
+  } else if (warp == kIssuerWarp) {
+    if (lane == 0 && p.stage_c) {
+      // ---- C issuer: TMA stores of the boxes the epilogue finished, TMA loads of the next
+      // tile's C into each box as soon as its store has left shared memory ----
+      const bool loads = p.beta != 0.f;
+      uint8_t* cs = smem + kStages * kStageBytes;
+      uint32_t rdy_ph = 0;      // per-box parity of the next ready[] completion
+      uint32_t rel = 0;         // boxes released at least once
+      uint32_t last_ph = 0;     // per-box parity of the latest release's cbox completion
+      auto release = [&](int m0n, int n0n, int j) {
+        if (rel & (1u << j)) last_ph ^= 1u << j;
+        rel |= 1u << j;
+        if (loads) {
+          mbar_arrive_expect_tx(&cbox[j], kBoxBytes);
+          tma_load_2d(cs + j * kBoxBytes, &tC, &cbox[j], n0n + 32 * j, m0n);
+        } else {
+          mbar_arrive(&cbox[j]);
+        }
+      };
+      auto n_boxes = [&](int n0) { return min(4, (p.N - n0 + 31) / 32); };
+      if (t_begin < t_end) {
+        int tm, tn;
+        tile_coords(p, t_begin, tm, tn);
+        const int nb0 = n_boxes(tn * BN);
+        for (int j = 0; j < nb0; ++j) release(tm * BM, tn * BN, j);
+      }
+      for (int t = t_begin; t < t_end; ++t) {
+        int tm, tn;
+        tile_coords(p, t, tm, tn);
+        const int m0 = tm * BM, n0 = tn * BN;
+        const int nbx = n_boxes(n0);
+        int nm0 = 0, nn0 = 0, nnb = 0;               // the next tile (nnb = 0: none)
+        if (t + 1 < t_end) {
+          int tm2, tn2;
+          tile_coords(p, t + 1, tm2, tn2);
+          nm0 = tm2 * BM;
+          nn0 = tn2 * BN;
+          nnb = n_boxes(nn0);
+        }
+        bool ok = true;
+        for (int j = 0; j < nbx; ++j) {
+          if (!mbar_wait_bounded(&ready[j], (rdy_ph >> j) & 1u, &abort_flag, info)) {
+            ok = false;
+            break;
+          }
+          rdy_ph ^= 1u << j;
+          tma_store_2d(&tC, cs + j * kBoxBytes, n0 + 32 * j, m0);
+          tma_store_commit();
+          if (j >= 1) {
+            tma_store_wait_read<1>();                // box j-1 has left shared memory
+            if (j - 1 < nnb) release(nm0, nn0, j - 1);
+          }
+        }
+        if (!ok) break;
+        tma_store_wait_read<0>();
+        for (int j = nbx - 1; j < nnb; ++j) release(nm0, nn0, j);
+      }
+      tma_store_wait_all();
+      if (loads)
+        for (int j = 0; j < 4; ++j)
+          if (rel & (1u << j)) mbar_drain_bounded(&cbox[j], (last_ph >> j) & 1u);
+    }
   } else if (p.stage_c) {
-    // ---- epilogue through shared memory (C loaded and stored by TMA) ----
+    // ---- epilogue through shared memory: fold TMEM, write the four 128 x 32 boxes (swizzled),
+    // hand each to the C issuer ----
     const int q = warp & 3;
     const int r = q * 32 + lane;                    // row within the tile (= TMEM lane)
+    const int et = threadIdx.x - 64;                // 0..127 within the epilogue group
     const uint32_t rsw = static_cast<uint32_t>(r & 7);
-    const bool st_thread = threadIdx.x == 64;       // issues the C loads and stores
     const bool loads = p.beta != 0.f;
+    const bool split = p.Cbig != nullptr;
     uint8_t* cs = smem + kStages * kStageBytes;
-    uint32_t cwait = 0;                             // per-box parity of the next c_full completion
-    uint32_t pend = 0;                              // boxes with a C load in flight (store thread)
+    uint32_t tok_ph = 0;                            // per-box parity of the next cbox completion
     auto n_boxes = [&](int n0) { return min(4, (p.N - n0 + 31) / 32); };
-    auto load_box = [&](int m0, int n0, int j) {
-      mbar_arrive_expect_tx(&c_full[j], kBoxBytes);
-      tma_load_2d(cs + j * kBoxBytes, &tC, &c_full[j], n0 + 32 * j, m0);
-      pend |= 1u << j;
-    };
-    if (st_thread && loads && t_begin < t_end) {
-      int tm, tn;
-      tile_coords(p, t_begin, tm, tn);
-      const int nbx = n_boxes(tn * BN);
-      for (int j = 0; j < nbx; ++j) load_box(tm * BM, tn * BN, j);
-    }
     int c = 0;
     for (int t = t_begin; t < t_end; ++t, ++c) {
       int tm, tn;
       tile_coords(p, t, tm, tn);
       const int m0 = tm * BM, n0 = tn * BN;
       const int nbx = n_boxes(n0);
-      int nm0 = 0, nn0 = 0, nnb = 0;                // the next tile (nnb = 0: none)
-      if (t + 1 < t_end) {
-        int tm2, tn2;
-        tile_coords(p, t + 1, tm2, tn2);
-        nm0 = tm2 * BM;
-        nn0 = tn2 * BN;
-        nnb = loads ? n_boxes(nn0) : 0;
-      }
       const int buf = c & 1;
       const bool ok = mbar_wait_bounded(&acc_full[buf], (c >> 1) & 1, &abort_flag, info);
       if (named_barrier_or(kEpiBarrier, 128, !ok || abort_flag)) break;
@@ -487,21 +537,15 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
-      const int row = m0 + r;
       bool stop = false;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (j < nbx && !stop) {
-          bool okc = true;
-          if (loads) {
-            okc = mbar_wait_bounded(&c_full[j], (cwait >> j) & 1u, &abort_flag, info);
-            if (okc) {
-              cwait ^= 1u << j;
-              pend &= ~(1u << j);
-            }
-          }
+        if (j < nbx) {
+          bool okc = !stop && mbar_wait_bounded(&cbox[j], (tok_ph >> j) & 1u, &abort_flag, info);
+          uint8_t* box = cs + j * kBoxBytes;
           if (okc) {
-            uint8_t* rowp = cs + j * kBoxBytes + r * 128;
+            tok_ph ^= 1u << j;
+            uint8_t* rowp = box + r * 128;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               float4* a = reinterpret_cast<float4*>(rowp + ((static_cast<uint32_t>(u) ^ rsw) << 4));
@@ -513,48 +557,46 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
                 v.z = fmaf(p.beta, o.z, v.z); v.w = fmaf(p.beta, o.w, v.w);
               }
               *a = v;
-              if (p.Cbig && row < p.M) {
-                const int col = n0 + j * 32 + 4 * u;
-                const float4 b = make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z),
-                                             tf32_round(v.w));
-                const float4 sm = make_float4(v.x - b.x, v.y - b.y, v.z - b.z, v.w - b.w);
-                float* bp = p.Cbig + static_cast<int64_t>(row) * p.ld_split + col;
-                float* sp = p.Csmall + static_cast<int64_t>(row) * p.ld_split + col;
-                if (col + 4 <= p.N) {
-                  *reinterpret_cast<float4*>(bp) = b;
-                  *reinterpret_cast<float4*>(sp) = sm;
-                } else {
-                  const float bb[4] = {b.x, b.y, b.z, b.w}, ss[4] = {sm.x, sm.y, sm.z, sm.w};
-                  for (int e = 0; e < 4 && col + e < p.N; ++e) {
-                    bp[e] = bb[e];
-                    sp[e] = ss[e];
+            }
+          }
+          stop = !okc;
+          if (split) {
+            // the tf32 split of the box, written row-contiguous from shared memory
+            stop = named_barrier_or(kEpiBarrier, 128, stop || abort_flag);
+            if (!stop) {
+#pragma unroll
+              for (int s2 = 0; s2 < 8; ++s2) {
+                const int f = et + 128 * s2;
+                const int br = f >> 3, u = f & 7;
+                const float4 v = *reinterpret_cast<const float4*>(
+                    box + br * 128 + ((static_cast<uint32_t>(u) ^ static_cast<uint32_t>(br & 7)) << 4));
+                const int row = m0 + br, col = n0 + 32 * j + 4 * u;
+                if (row < p.M) {
+                  const float4 bg = make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z),
+                                                tf32_round(v.w));
+                  const float4 sm = make_float4(v.x - bg.x, v.y - bg.y, v.z - bg.z, v.w - bg.w);
+                  float* bp = p.Cbig + static_cast<int64_t>(row) * p.ld_split + col;
+                  float* sp = p.Csmall + static_cast<int64_t>(row) * p.ld_split + col;
+                  if (col + 4 <= p.N) {
+                    *reinterpret_cast<float4*>(bp) = bg;
+                    *reinterpret_cast<float4*>(sp) = sm;
+                  } else {
+                    const float bb[4] = {bg.x, bg.y, bg.z, bg.w}, ss[4] = {sm.x, sm.y, sm.z, sm.w};
+                    for (int e = 0; e < 4 && col + e < p.N; ++e) {
+                      bp[e] = bb[e];
+                      sp[e] = ss[e];
+                    }
                   }
                 }
               }
             }
           }
-          fence_proxy_async_smem();
-          stop = named_barrier_or(kEpiBarrier, 128, !okc || abort_flag);
-          if (!stop && st_thread) {
-            tma_store_2d(&tC, cs + j * kBoxBytes, n0 + 32 * j, m0);
-            tma_store_commit();
-            if (j >= 1) {
-              tma_store_wait_read<1>();             // box j-1 has left shared memory
-              if (j - 1 < nnb) load_box(nm0, nn0, j - 1);
-            }
+          if (!stop) {
+            fence_proxy_async_smem();
+            mbar_arrive(&ready[j]);
           }
         }
       }
-      if (stop) break;
-      if (st_thread) {
-        tma_store_wait_read<0>();
-        for (int j = nbx - 1; j < nnb; ++j) load_box(nm0, nn0, j);
-      }
-    }
-    if (st_thread) {
-      tma_store_wait_all();
-      for (int j = 0; j < 4; ++j)
-        if (pend & (1u << j)) mbar_drain_bounded(&c_full[j], (cwait >> j) & 1u);
     }
   } else {
     const int q = warp & 3;
