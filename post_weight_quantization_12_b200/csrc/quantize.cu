@@ -194,50 +194,86 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   }
   float inv_s = 1.f / s;
 
+  // Columns go in sub-blocks of four, 32t + 4o .. 32t + 4o + 3, all held by lane o of the row.
+  // Every lane of the row takes the four current values from their owner and quantizes them
+  // itself, applying each column's error to the sub-block's later columns in registers; then
+  // each lane applies the four errors to its own later columns (a rank-4 update whose FMAs run in
+  // the same order as four rank-1 updates). Only the owner keeps the results.
+  int gcnt = 0;                             // position in the current group (group_mode 1)
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
-    for (int o = 0; o < kTPR; ++o) {        // owner lane of columns 32t + 4o .. 32t + 4o + 3
+    for (int o = 0; o < kTPR; ++o) {
+      const int j0 = 32 * t + 4 * o;
+      if (j0 >= nb) break;
+      const bool own = (sub == o);
+      float w4[4], e4[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) w4[u] = __shfl_sync(0xffffffffu, v[4 * t + u], base_lane + o);
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int j = 32 * t + 4 * o + u;
-        const int kk = 4 * t + u;           // register slot of column j in its owner lane
+        const int j = j0 + u;
+        e4[u] = 0.f;
         if (j < nb) {
-          if (group_mode == 1 && (j % group) == 0) {
-            float lo = 0.f, hi = 0.f;
+          if (group_mode == 1) {
+            if (gcnt == 0) {
+              float lo = 0.f, hi = 0.f;
+              if (group <= 4) {
+                // the group lies inside this sub-block, whose current values every lane holds
 #pragma unroll
-            for (int k = 0; k < CPL; ++k) {
-              const int c = colof(k);
-              if (c >= j && c < j + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
-            }
+                for (int u2 = 0; u2 < 4; ++u2)
+                  if (u2 >= u && u2 < u + group && j0 + u2 < nb) {
+                    lo = fminf(lo, w4[u2]);
+                    hi = fmaxf(hi, w4[u2]);
+                  }
+              } else {
+                // the group starts at this sub-block (u == 0): the row's lanes hold it
 #pragma unroll
-            for (int off = kTPR / 2; off > 0; off >>= 1) {
-              lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-              hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+                for (int k = 0; k < CPL; ++k) {
+                  const int c = colof(k);
+                  if (c >= j && c < j + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
+                }
+#pragma unroll
+                for (int off = kTPR / 2; off > 0; off >>= 1) {
+                  lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+                  hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+                }
+              }
+              grid_params(lo, hi, maxq, s, z);
+              inv_s = 1.f / s;
+              if (valid && sub == 0) {
+                const int gi = (b0 + j) / group;
+                scales[row * G + gi] = s;
+                zeros[row * G + gi] = static_cast<uint8_t>(z);
+              }
             }
-            grid_params(lo, hi, maxq, s, z);
-            inv_s = 1.f / s;
-            if (valid && sub == 0) {
-              const int gi = (b0 + j) / group;
-              scales[row * G + gi] = s;
-              zeros[row * G + gi] = static_cast<uint8_t>(z);
-            }
+            gcnt = (gcnt + 1 == group) ? 0 : gcnt + 1;
           }
-          const float w = __shfl_sync(0xffffffffu, v[kk], base_lane + o);
+          const float w = w4[u];
           const float q = fminf(fmaxf(rint_quot(w, s, inv_s) + z, 0.f), maxq);
           const float wh = __fmul_rn(s, q - z);
           const float e = __fmul_rn(__fsub_rn(w, wh), inv_d[j]);
-          const bool own = (sub == o);
-          v[kk] = own ? wh : v[kk];
-          q8[kk] = own ? static_cast<uint8_t>(q) : q8[kk];
-          err[kk] = own ? e : err[kk];
+          e4[u] = e;
+          v[4 * t + u] = own ? wh : v[4 * t + u];
+          q8[4 * t + u] = own ? static_cast<uint8_t>(q) : q8[4 * t + u];
+          err[4 * t + u] = own ? e : err[4 * t + u];
 #pragma unroll
-          for (int t2 = 0; t2 < NT; ++t2) {
-            const float4 r4 = *reinterpret_cast<const float4*>(&Rz[j][32 * t2 + 4 * sub]);
-            v[4 * t2 + 0] = fmaf(-e, r4.x, v[4 * t2 + 0]);
-            v[4 * t2 + 1] = fmaf(-e, r4.y, v[4 * t2 + 1]);
-            v[4 * t2 + 2] = fmaf(-e, r4.z, v[4 * t2 + 2]);
-            v[4 * t2 + 3] = fmaf(-e, r4.w, v[4 * t2 + 3]);
-          }
+          for (int u2 = u + 1; u2 < 4; ++u2) w4[u2] = fmaf(-e, Rz[j][j0 + u2], w4[u2]);
+        }
+      }
+#pragma unroll
+      for (int t2 = t; t2 < NT; ++t2) {
+        // the owner's own four columns of group t are final already
+        const bool skip = (t2 == t) && own;
+        float4 r[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) r[u] = *reinterpret_cast<const float4*>(&Rz[j0 + u][32 * t2 + 4 * sub]);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float c = skip ? 0.f : e4[u];
+          v[4 * t2 + 0] = fmaf(-c, r[u].x, v[4 * t2 + 0]);
+          v[4 * t2 + 1] = fmaf(-c, r[u].y, v[4 * t2 + 1]);
+          v[4 * t2 + 2] = fmaf(-c, r[u].z, v[4 * t2 + 2]);
+          v[4 * t2 + 3] = fmaf(-c, r[u].w, v[4 * t2 + 3]);
         }
       }
     }
