@@ -60,6 +60,23 @@ __device__ __forceinline__ float load_w<__nv_bfloat16>(const __nv_bfloat16* p) {
   return __bfloat162float(*p);
 }
 
+// bf16 rows of 8-element chunks (16-byte loads, two float4 stores); cols % 8 == 0, ldw % 8 == 0
+__global__ void convert_bf16_vec_kernel(const __nv_bfloat16* __restrict__ W, int64_t ldw,
+                                        float* __restrict__ Wh, int64_t rows, int64_t cols) {
+  const int64_t c8 = cols / 8, total = rows * c8;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = e / c8, c = 8 * (e - r * c8);
+    const uint4 raw = *reinterpret_cast<const uint4*>(W + r * ldw + c);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+    const float2 f0 = __bfloat1622float2(h[0]), f1 = __bfloat1622float2(h[1]);
+    const float2 f2 = __bfloat1622float2(h[2]), f3 = __bfloat1622float2(h[3]);
+    float4* dst = reinterpret_cast<float4*>(Wh + r * cols + c);
+    dst[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
+    dst[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
+  }
+}
+
 template <typename T>
 __global__ void convert_kernel(const T* __restrict__ W, int64_t ldw, float* __restrict__ Wh,
                                int64_t rows, int64_t cols) {
@@ -109,7 +126,8 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
                    int b0, int nb, int bits, int group, int group_mode, int gi_fixed,
                    float* __restrict__ scales, uint8_t* __restrict__ zeros, int G,
                    uint8_t* __restrict__ codes, float* __restrict__ Eb, float* __restrict__ Es,
-                   float* __restrict__ err_sq) {
+                   float* __restrict__ err_sq, float* __restrict__ Rb_out,
+                   float* __restrict__ Rs_out, int64_t nrest) {
   constexpr int NT = B / 32;       // float4 groups per lane
   constexpr int CPL = 4 * NT;      // columns per lane
   extern __shared__ __align__(16) float qsm[];
@@ -152,6 +170,20 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   }
   for (int i = threadIdx.x; i < B; i += blockDim.x)
     inv_d[i] = (i < nb) ? 1.f / R[(b0 + i) * cols + b0 + i] : 0.f;
+  // the tf32 split of R[b0 : b0 + nb, b1 : cols] for the trailing product that follows this block,
+  // spread over the whole grid (rows 16-byte aligned: cols % 4 == 0, b1 % 4 == 0)
+  if (nrest > 0) {
+    const int64_t b1 = b0 + nb, n4 = nrest / 4, total = nb * n4;
+    for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+      const int64_t i = e / n4, c = b1 + 4 * (e - i * n4);
+      const float4 x = *reinterpret_cast<const float4*>(R + (b0 + i) * cols + c);
+      const float4 bg = make_float4(tf32_rna_q(x.x), tf32_rna_q(x.y), tf32_rna_q(x.z), tf32_rna_q(x.w));
+      *reinterpret_cast<float4*>(Rb_out + i * cols + c) = bg;
+      *reinterpret_cast<float4*>(Rs_out + i * cols + c) =
+          make_float4(x.x - bg.x, x.y - bg.y, x.z - bg.z, x.w - bg.w);
+    }
+  }
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
@@ -331,7 +363,8 @@ template <int B>
 static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, const float* R, int b0,
                                       int nb, int bits, int group, int group_mode, int gi_fixed,
                                       float* scales, uint8_t* zeros, int G, uint8_t* codes,
-                                      float* Eb, float* Es, float* err_sq, cudaStream_t stream) {
+                                      float* Eb, float* Es, float* err_sq, float* Rb, float* Rs,
+                                      int64_t nrest, cudaStream_t stream) {
   const int rows_per_cta = 128 / kTPR;
   const int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
   constexpr int smem = (B * B + B) * 4;
@@ -344,7 +377,7 @@ static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, con
   }
   column_loop_kernel<B><<<static_cast<unsigned>(grid), 128, smem, stream>>>(
       Wh, rows, cols, R, b0, nb, bits, group, group_mode, gi_fixed, scales, zeros, G, codes, Eb,
-      Es, err_sq);
+      Es, err_sq, Rb, Rs, nrest);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }
@@ -363,7 +396,11 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
   const int G = group > 0 ? static_cast<int>(cols / group) : 1;
   const int64_t total = rows * cols;
   const int cgrid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 8 * 148));
-  if (w_dtype == GPTQ_BF16)
+  if (w_dtype == GPTQ_BF16 && cols % 8 == 0 && ldw % 8 == 0 &&
+      (reinterpret_cast<uintptr_t>(W) & 15) == 0)
+    convert_bf16_vec_kernel<<<std::min<int64_t>((total / 8 + 255) / 256, 8 * 148), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(W), ldw, Wh, rows, cols);
+  else if (w_dtype == GPTQ_BF16)
     convert_kernel<__nv_bfloat16><<<cgrid, 256, 0, stream>>>(
         static_cast<const __nv_bfloat16*>(W), ldw, Wh, rows, cols);
   else
@@ -382,7 +419,8 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
   for (int64_t b0 = 0; b0 < cols; b0 += block) {
     const int nb = static_cast<int>(cols - b0 < block ? cols - b0 : block);
     int mode = 0, gi = 0;
-    if (group > 0 && group % block == 0) {
+    const int64_t b1 = b0 + nb, nrest = cols - b1;
+    if (group > 0 && group % block == 0 && group != block) {
       gi = static_cast<int>(b0 / group);
       if (b0 % group == 0) {
         params_kernel<<<pgrid, 256, 0, stream>>>(Wh, rows, cols, b0, group, bits, scales, zeros, G,
@@ -393,28 +431,28 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
     } else if (group > 0) {
       mode = 1;
     }
+    // the column loop also writes the tf32 split of R[b0:b1, b1:] into (Rb, Rs) for S8
     gptq_status st;
     switch (block) {
       case 32:
         st = launch_column_loop<32>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group, mode,
-                                    gi, scales, zeros, G, codes, Eb, Es, err_sq, stream);
+                                    gi, scales, zeros, G, codes, Eb, Es, err_sq, Rb, Rs, nrest,
+                                    stream);
         break;
       case 64:
         st = launch_column_loop<64>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group, mode,
-                                    gi, scales, zeros, G, codes, Eb, Es, err_sq, stream);
+                                    gi, scales, zeros, G, codes, Eb, Es, err_sq, Rb, Rs, nrest,
+                                    stream);
         break;
       default:
         st = launch_column_loop<128>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group,
-                                     mode, gi, scales, zeros, G, codes, Eb, Es, err_sq, stream);
+                                     mode, gi, scales, zeros, G, codes, Eb, Es, err_sq, Rb, Rs,
+                                     nrest, stream);
         break;
     }
     if (st != GPTQ_OK) return st;
-    const int64_t b1 = b0 + nb;
     if (b1 < cols) {
       // S8: W[:, b1:] -= E * R[b0:b1, b1:] on the tensor cores (3xTF32)
-      const int64_t nrest = cols - b1;
-      st = launch_split_tf32(R + b0 * cols + b1, cols, nb, nrest, Rb + b1, Rs + b1, cols, stream);
-      if (st != GPTQ_OK) return st;
       TcGemmArgs g{Eb, Es, Rb + b1, Rs + b1, block, cols, 0, 1,
                    static_cast<int>(rows), static_cast<int>(nrest), nb, -1.f, 1.f, 0, 0, 0,
                    Wh + b1, cols, nullptr, nullptr, 0, info};
