@@ -7,12 +7,12 @@
 // (W[:, B:] -= E R[B, B:]); the design table and the blog's "Group-wise quantization"
 // (asymmetric uniform grid per row or per group).
 //
-// Column loop layout: 8 consecutive lanes own one weight row; lane t of the row holds columns
-// [t * B/8, (t + 1) * B/8) of the current block in registers. The block's B x B corner of R sits
-// in shared memory with its diagonal and lower part replaced by zeros, so the in-block update
-// w[c] -= e * R[j][c] needs no mask (columns at or before j are left untouched). Every lane of a
-// row computes the same code for column j from the value broadcast by its owner lane, so no
-// further communication is needed per column.
+// Column loop layout: TPR consecutive lanes (16, or 8 for 32-column blocks) own one weight row and
+// hold the current block's values of that row in registers, four consecutive columns per lane per
+// stretch of 4 * TPR columns. The block's B x B corner of R sits in shared memory with its
+// diagonal and lower part replaced by zeros, so updates need no mask (columns at or before j are
+// left untouched). Every lane of a row computes the same codes for a sub-block of four columns
+// from values broadcast by their owner lane, so one exchange serves four columns.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -22,7 +22,6 @@
 
 namespace gptq {
 
-constexpr int kTPR = 8;  // lanes per weight row
 
 // tf32 rounding, for the (big, small) operand split of the trailing product
 __device__ __forceinline__ float tf32_rna_q(float x) {
@@ -116,19 +115,20 @@ __global__ void params_kernel(const float* __restrict__ Wh, int64_t rows, int64_
 // One block of B columns [b0, b0 + nb) for every row.
 //   group_mode: 0 = grid given per row (scales[row*G + gi_fixed]);
 //               1 = groups of `group` columns inside the block, grids computed here.
-// Lane `sub` of a row holds, in registers, the columns 32*t + 4*sub + u (t < B/32, u < 4): the 8
-// lanes of a row together cover each 32-column stretch with one float4 each, so their reads of a
-// row of R and their loads/stores of W, E and codes are contiguous 128-byte segments (no shared
-// memory bank conflicts, coalesced global accesses).
-template <int B>
-__global__ void __launch_bounds__(128)
+// Lane `sub` of a row holds, in registers, the columns S*t + 4*sub + u (S = 4 TPR, t < B/S,
+// u < 4): the TPR lanes of a row together cover each S-column stretch with one float4 each, so
+// their reads of a row of R and their loads/stores of W, E and codes are contiguous segments (no
+// shared memory bank conflicts, coalesced global accesses).
+template <int B, int TPR, int THREADS>
+__global__ void __launch_bounds__(THREADS)
 column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const float* __restrict__ R,
                    int b0, int nb, int bits, int group, int group_mode, int gi_fixed,
                    float* __restrict__ scales, uint8_t* __restrict__ zeros, int G,
                    uint8_t* __restrict__ codes, float* __restrict__ Eb, float* __restrict__ Es,
                    float* __restrict__ err_sq, float* __restrict__ Rb_out,
                    float* __restrict__ Rs_out, int64_t nrest) {
-  constexpr int NT = B / 32;       // float4 groups per lane
+  constexpr int S = 4 * TPR;       // columns covered by one float4 from each lane of a row
+  constexpr int NT = B / S;        // float4 groups per lane
   constexpr int CPL = 4 * NT;      // columns per lane
   extern __shared__ __align__(16) float qsm[];
   float (*Rz)[B] = reinterpret_cast<float (*)[B]>(qsm);
@@ -136,11 +136,11 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   // the block's corner of R with its diagonal and lower part zeroed; every load in flight at once
   // (rows are 16-byte aligned: cols % 4 == 0, b0 % 4 == 0)
   {
-    constexpr int PER = B * B / 4 / 128;  // float4 per thread
+    constexpr int PER = B * B / 4 / THREADS;  // float4 per thread
     float4 buf[PER];
 #pragma unroll
     for (int p = 0; p < PER; ++p) {
-      const int e = threadIdx.x + p * 128;
+      const int e = threadIdx.x + p * THREADS;
       const int i = (4 * e) / B, j = (4 * e) % B;
       float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
       if (i < nb) {
@@ -158,7 +158,7 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
     }
 #pragma unroll
     for (int p = 0; p < PER; ++p) {
-      const int e = threadIdx.x + p * 128;
+      const int e = threadIdx.x + p * THREADS;
       const int i = (4 * e) / B, j = (4 * e) % B;
       float4 q = buf[p];
       q.x = (j + 0 > i) ? q.x : 0.f;
@@ -174,31 +174,47 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   // spread over the whole grid (rows 16-byte aligned: cols % 4 == 0, b1 % 4 == 0)
   if (nrest > 0) {
     const int64_t b1 = b0 + nb, n4 = nrest / 4, total = nb * n4;
-    for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-         e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-      const int64_t i = e / n4, c = b1 + 4 * (e - i * n4);
-      const float4 x = *reinterpret_cast<const float4*>(R + (b0 + i) * cols + c);
-      const float4 bg = make_float4(tf32_rna_q(x.x), tf32_rna_q(x.y), tf32_rna_q(x.z), tf32_rna_q(x.w));
-      *reinterpret_cast<float4*>(Rb_out + i * cols + c) = bg;
-      *reinterpret_cast<float4*>(Rs_out + i * cols + c) =
-          make_float4(x.x - bg.x, x.y - bg.y, x.z - bg.z, x.w - bg.w);
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * THREADS;
+    for (int64_t e0 = blockIdx.x * static_cast<int64_t>(THREADS) + threadIdx.x; e0 < total;
+         e0 += 4 * stride) {
+      float4 x[4];                         // four loads in flight
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t e = e0 + u * stride;
+        if (e < total) {
+          const int64_t i = e / n4, c = b1 + 4 * (e - i * n4);
+          x[u] = *reinterpret_cast<const float4*>(R + (b0 + i) * cols + c);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int64_t e = e0 + u * stride;
+        if (e < total) {
+          const int64_t i = e / n4, c = b1 + 4 * (e - i * n4);
+          const float4 bg = make_float4(tf32_rna_q(x[u].x), tf32_rna_q(x[u].y),
+                                        tf32_rna_q(x[u].z), tf32_rna_q(x[u].w));
+          *reinterpret_cast<float4*>(Rb_out + i * cols + c) = bg;
+          *reinterpret_cast<float4*>(Rs_out + i * cols + c) =
+              make_float4(x[u].x - bg.x, x[u].y - bg.y, x[u].z - bg.z, x[u].w - bg.w);
+        }
+      }
     }
   }
   __syncthreads();
 
   const int lane = threadIdx.x & 31;
-  const int sub = lane & (kTPR - 1);          // position within the row's lane group
-  const int base_lane = lane & ~(kTPR - 1);
-  const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x / kTPR) + threadIdx.x / kTPR;
+  const int sub = lane & (TPR - 1);           // position within the row's lane group
+  const int base_lane = lane & ~(TPR - 1);
+  const int64_t row = blockIdx.x * static_cast<int64_t>(THREADS / TPR) + threadIdx.x / TPR;
   const bool valid = row < rows;
-  auto colof = [&](int k) { return 32 * (k >> 2) + 4 * sub + (k & 3); };  // block column of v[k]
+  auto colof = [&](int k) { return S * (k >> 2) + 4 * sub + (k & 3); };  // block column of v[k]
 
   float v[CPL];
   uint8_t q8[CPL];
   float err[CPL];
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
-    const int c = 32 * t + 4 * sub;
+    const int c = S * t + 4 * sub;
     float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
     if (valid) {
       const float* src = Wh + row * cols + b0 + c;
@@ -234,8 +250,8 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   int gcnt = 0;                             // position in the current group (group_mode 1)
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
-    for (int o = 0; o < kTPR; ++o) {
-      const int j0 = 32 * t + 4 * o;
+    for (int o = 0; o < TPR; ++o) {
+      const int j0 = S * t + 4 * o;
       if (j0 >= nb) break;
       const bool own = (sub == o);
       float w4[4], e4[4];
@@ -265,7 +281,7 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
                   if (c >= j && c < j + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
                 }
 #pragma unroll
-                for (int off = kTPR / 2; off > 0; off >>= 1) {
+                for (int off = TPR / 2; off > 0; off >>= 1) {
                   lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
                   hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
                 }
@@ -298,7 +314,7 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
         const bool skip = (t2 == t) && own;
         float4 r[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) r[u] = *reinterpret_cast<const float4*>(&Rz[j0 + u][32 * t2 + 4 * sub]);
+        for (int u = 0; u < 4; ++u) r[u] = *reinterpret_cast<const float4*>(&Rz[j0 + u][S * t2 + 4 * sub]);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const float c = skip ? 0.f : e4[u];
@@ -315,11 +331,11 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
 #pragma unroll
   for (int k = 0; k < CPL; ++k) sq = fmaf(err[k], err[k], sq);
 #pragma unroll
-  for (int off = kTPR / 2; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
+  for (int off = TPR / 2; off > 0; off >>= 1) sq += __shfl_xor_sync(0xffffffffu, sq, off);
   if (!valid) return;
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
-    const int c = 32 * t + 4 * sub;
+    const int c = S * t + 4 * sub;
     float* wd = Wh + row * cols + b0 + c;
     uint8_t* cd = codes + row * cols + b0 + c;
     float* eb = Eb + row * B + c;
@@ -365,17 +381,21 @@ static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, con
                                       float* scales, uint8_t* zeros, int G, uint8_t* codes,
                                       float* Eb, float* Es, float* err_sq, float* Rb, float* Rs,
                                       int64_t nrest, cudaStream_t stream) {
-  const int rows_per_cta = 128 / kTPR;
+  // 16 lanes per row for blocks of 64 or 128 columns (more warps, less per-lane update work),
+  // 8 for 32 columns
+  constexpr int TPR = B >= 64 ? 16 : 8;
+  constexpr int THREADS = B >= 64 ? 256 : 128;
+  const int rows_per_cta = THREADS / TPR;
   const int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
   constexpr int smem = (B * B + B) * 4;
   static bool attr_done = false;
   if (!attr_done) {
-    if (cudaFuncSetAttribute(column_loop_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    if (cudaFuncSetAttribute(column_loop_kernel<B, TPR, THREADS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return GPTQ_ECUDA;
     attr_done = true;
   }
-  column_loop_kernel<B><<<static_cast<unsigned>(grid), 128, smem, stream>>>(
+  column_loop_kernel<B, TPR, THREADS><<<static_cast<unsigned>(grid), THREADS, smem, stream>>>(
       Wh, rows, cols, R, b0, nb, bits, group, group_mode, gi_fixed, scales, zeros, G, codes, Eb,
       Es, err_sq, Rb, Rs, nrest);
   count_launch();
