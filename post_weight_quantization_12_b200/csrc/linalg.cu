@@ -188,9 +188,10 @@ reverse_to_upper_kernel(float* R, const float* Vb, const float* Vs, int64_t n) {
 // S3/S5 diagonal block: Cholesky of A[k0:k0+nb, k0:k0+nb] on chip (lower; the block's strict upper
 // part is zeroed in A when store_l is set) and the tf32 split of its triangular inverse into
 // (Db, Ds) with ld ldd. Blocked by 32-column pieces; for each piece kb:
-//  F  warp 0 factors the piece and builds its inverse in the same loop, four columns per step
-//     (factor_piece4).
-//     Meanwhile warps 1-15 form the block's inverse row blocks,
+//  F  warps 0-3 factor the piece and build its inverse in the same loop, four columns per step
+//     (factor_piece4_mw).
+//     Meanwhile warps 4-15 finish the previous piece's trailing update beyond this piece's
+//     columns and form the block's inverse row blocks,
 //     X[b][j] = -X[b][b] * sum_m L[b][m] X[m][j]: the sum for row block kb and the product with
 //     X[kb-1][kb-1] for row block kb-1.
 //  S  rows below the piece: L21 = A21 X_kk^T, 4 x 4 register tiles, written transposed into PT;
@@ -202,8 +203,8 @@ reverse_to_upper_kernel(float* R, const float* Vb, const float* Vs, int64_t n) {
 // ------------------------------------------------------------------------------------------------
 namespace la {
 constexpr int kLdt = 100;      // PT / OT row: 96 entries + pad, a multiple of 4 for float4 access
-constexpr int kInverseBar = 1;
-constexpr int kInverseThreads = kDiagThreads - 32;
+constexpr int kInverseBar = 1, kFactorBar = 2;
+constexpr int kInverseThreads = kDiagThreads - 128;
 }
 
 // First half of row block b of the inverse: OT[r][j] = sum_m L[32b + r][m] X[m][j], j < 32b, over
@@ -260,80 +261,115 @@ __device__ __forceinline__ void inverse_row_product(float* X, const float* OT, i
     for (int v = 0; v < 4; ++v) X[(r0 + u) * LD + 4 * jg + v] = -acc[u][v];
 }
 
-// Factor and invert one 32 x 32 piece in one warp, four columns per step. Lane l is row l; e[k]
-// holds L[l][k] for k < l (the factor's row) and the running sum for X[k][l] for k > l (the
-// inverse's column, X[j][t] = (delta_jt - sum_{m<j} L[j][m] X[m][t]) / L[j][j]); the diagonal pair
-// L[l][l], X[l][l] ends in ldiag / xdiag. Per step every lane factors the step's 4 x 4 diagonal
-// block itself (broadcast by shuffles), solves its own four entries of L or X, and applies the
-// four new columns to its remaining registers: entries of L take -L[l][j] L[k][j], entries of X
-// take L[k][j] X[j][l], so one FMA per register and column serves both. `col` holds two 32-entry
-// buffers. A pivot that is not positive is replaced by 1 and its index goes to badj.
-__device__ __forceinline__ void factor_piece4(float (&e)[32], float& ldiag, float& xdiag, int& badj,
-                                              float4* col, int lane) {
+// Factor and invert one 32 x 32 piece, four columns per step, on warps 0-3. Lane l is row l; each
+// register holds L[l][k] for k < l (the factor's row) or the running sum for X[k][l] for k > l (the
+// inverse's column, X[j][t] = (delta_jt - sum_{m<j} L[j][m] X[m][t]) / L[j][j]); the diagonal
+// pair L[l][l], X[l][l] ends in ldiag / xdiag. Per step the owning warp factors the step's 4 x 4
+// diagonal block itself (broadcast by shuffles) and solves every row's four entries of L or X;
+// entries of L then take -L[l][j] L[k][j] and entries of X take L[k][j] X[j][l], so one FMA per
+// register and column serves both. A pivot that is not positive is replaced by 1 and its index
+// goes to badj. Warp w keeps columns 8w .. 8w+7 of every row in e[0..7]; step t (columns
+// 4t .. 4t+3) belongs to warp t/2, which publishes every row's entries of L (A4) and of X (X4) for
+// the step; after a barrier of the four warps each warp applies them to its later columns.
+// ldiag / xdiag are valid in the warp that owns column `lane`.
+__device__ __forceinline__ void factor_piece4_mw(float (&e)[8], float& ldiag, float& xdiag,
+                                                 int& badj, float4* A4, float4* X4, int warp,
+                                                 int lane) {
 #pragma unroll
   for (int t = 0; t < 8; ++t) {
-    const int j = 4 * t;
-    float b[4][4];
+    const int j = 4 * t, q0 = (t & 1) * 4;
+    if (warp == (t >> 1)) {
+      float b[4][4];
 #pragma unroll
-    for (int p = 0; p < 4; ++p)
+      for (int p = 0; p < 4; ++p)
 #pragma unroll
-      for (int q = 0; q <= p; ++q) b[p][q] = __shfl_sync(0xffffffffu, e[j + q], j + p);
-    float lb[4][4], r[4];
+        for (int q = 0; q <= p; ++q) b[p][q] = __shfl_sync(0xffffffffu, e[q0 + q], j + p);
+      float lb[4][4], r[4];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      float d = b[q][q];
+      for (int q = 0; q < 4; ++q) {
+        float d = b[q][q];
 #pragma unroll
-      for (int s = 0; s < q; ++s) d = fmaf(-lb[q][s], lb[q][s], d);
-      const bool ok = d > 0.f && d < INFINITY;
-      r[q] = ok ? rsqrtf(d) : 1.f;
-      lb[q][q] = ok ? d * r[q] : 1.f;
-      badj = (!ok && badj == 32) ? j + q : badj;
+        for (int s = 0; s < q; ++s) d = fmaf(-lb[q][s], lb[q][s], d);
+        const bool ok = d > 0.f && d < INFINITY;
+        r[q] = ok ? rsqrtf(d) : 1.f;
+        lb[q][q] = ok ? d * r[q] : 1.f;
+        badj = (!ok && badj == 32) ? j + q : badj;
 #pragma unroll
-      for (int p = q + 1; p < 4; ++p) {
-        float v = b[p][q];
+        for (int p = q + 1; p < 4; ++p) {
+          float v = b[p][q];
 #pragma unroll
-        for (int s = 0; s < q; ++s) v = fmaf(-lb[p][s], lb[q][s], v);
-        lb[p][q] = v * r[q];
+          for (int s = 0; s < q; ++s) v = fmaf(-lb[p][s], lb[q][s], v);
+          lb[p][q] = v * r[q];
+        }
       }
+      float a[4], x[4];                    // L[lane][j+q] and X[j+q][lane]
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int k = j + q;
+        float sa = e[q0 + q], sx = -e[q0 + q];
+#pragma unroll
+        for (int s = 0; s < q; ++s) {
+          sa = fmaf(-a[s], lb[q][s], sa);
+          sx = fmaf(-lb[q][s], x[s], sx);
+        }
+        if (lane > k) {
+          a[q] = sa * r[q];
+          x[q] = 0.f;
+          e[q0 + q] = a[q];
+        } else if (lane == k) {
+          a[q] = lb[q][q];
+          x[q] = r[q];
+          ldiag = lb[q][q];
+          xdiag = r[q];
+        } else {
+          a[q] = 0.f;
+          x[q] = sx * r[q];
+          e[q0 + q] = x[q];
+        }
+      }
+      A4[t * 32 + lane] = make_float4(a[0], a[1], a[2], a[3]);
+      X4[t * 32 + lane] = make_float4(x[0], x[1], x[2], x[3]);
     }
-    float a[4], x[4];                      // L[lane][j+q] and X[j+q][lane]
+    named_barrier_or(la::kFactorBar, 128, false);
+    if (warp >= (t >> 1)) {
+      const float4 a4 = A4[t * 32 + lane], x4 = X4[t * 32 + lane];
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int k = j + q;
-      float sa = e[k], sx = -e[k];
-#pragma unroll
-      for (int s = 0; s < q; ++s) {
-        sa = fmaf(-a[s], lb[q][s], sa);
-        sx = fmaf(-lb[q][s], x[s], sx);
+      for (int q = 0; q < 8; ++q) {
+        const int k = 8 * warp + q;
+        if (k > j + 3) {
+          const float4 c = A4[t * 32 + k];
+          const bool fac = lane >= k;
+          e[q] = fmaf(c.x, fac ? -a4.x : x4.x, e[q]);
+          e[q] = fmaf(c.y, fac ? -a4.y : x4.y, e[q]);
+          e[q] = fmaf(c.z, fac ? -a4.z : x4.z, e[q]);
+          e[q] = fmaf(c.w, fac ? -a4.w : x4.w, e[q]);
+        }
       }
-      if (lane > k) {
-        a[q] = sa * r[q];
-        x[q] = 0.f;
-        e[k] = a[q];
-      } else if (lane == k) {
-        a[q] = lb[q][q];
-        x[q] = r[q];
-        ldiag = lb[q][q];
-        xdiag = r[q];
-      } else {
-        a[q] = 0.f;
-        x[q] = sx * r[q];
-        e[k] = x[q];
-      }
-    }
-    float4* cb = col + (t & 1) * 32;
-    cb[lane] = make_float4(a[0], a[1], a[2], a[3]);
-    __syncwarp();
-#pragma unroll
-    for (int k = j + 4; k < 32; ++k) {
-      const float4 c = cb[k];
-      const bool fac = lane >= k;
-      e[k] = fmaf(c.x, fac ? -a[0] : x[0], e[k]);
-      e[k] = fmaf(c.y, fac ? -a[1] : x[1], e[k]);
-      e[k] = fmaf(c.z, fac ? -a[2] : x[2], e[k]);
-      e[k] = fmaf(c.w, fac ? -a[3] : x[3], e[k]);
     }
   }
+}
+
+// One lower 4 x 4 tile of the trailing update A22 -= L21 L21^T inside the diagonal block: rows
+// c0 + 32 + 4 bi .., columns c0 + 32 + 4 bl .. (bl <= bi), the panel L21 read transposed from PT.
+__device__ __forceinline__ void trailing_tile(const float* PT, float* L, int c0, int bi, int bl) {
+  constexpr int LD = la::kLd, LDT = la::kLdt;
+  float acc[4][4] = {};
+#pragma unroll 8
+  for (int m = 0; m < 32; ++m) {
+    const float4 a4 = *reinterpret_cast<const float4*>(PT + m * LDT + 4 * bi);
+    const float4 b4 = *reinterpret_cast<const float4*>(PT + m * LDT + 4 * bl);
+    const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
+  }
+  const int i0 = c0 + 32 + 4 * bi, l0 = c0 + 32 + 4 * bl;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int v = 0; v < 4; ++v)
+      if (l0 + v <= i0 + u) L[(i0 + u) * LD + l0 + v] -= acc[u][v];
 }
 
 __global__ void __launch_bounds__(la::kDiagThreads)
@@ -345,7 +381,8 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
   float* X = sm + NB * LD;
   float* PT = sm + 2 * NB * LD;    // [32][LDT]: the panel below the piece, transposed
   float* OT = PT + 32 * LDT;       // 2 x [32][LDT]: partial sums of inverse row blocks
-  __shared__ float4 col4[64];     // four new columns per step, double-buffered
+  __shared__ float4 stepA[256];    // per factor step: every row's four entries of L
+  __shared__ float4 stepX[256];    // per factor step: every row's four entries of X
   __shared__ int bad;              // first pivot that was not positive (INT_MAX: none)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) bad = INT_MAX;
@@ -383,23 +420,37 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
 #pragma unroll 1
   for (int kb = 0; kb < 4; ++kb) {
     const int c0 = kb * 32;
-    if (warp == 0) {
-      // ---- F: factor and invert the piece ----
-      float e[32];
+    if (warp < 4) {
+      // ---- F: factor and invert the piece (warps 0-3) ----
+      float e[8];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) e[k] = (k <= lane) ? L[(c0 + lane) * LD + c0 + k] : 0.f;
+      for (int q = 0; q < 8; ++q) {
+        const int k = 8 * warp + q;
+        e[q] = (k <= lane) ? L[(c0 + lane) * LD + c0 + k] : 0.f;
+      }
       float ldiag = 1.f, xdiag = 1.f;
       int badj = 32;
-      factor_piece4(e, ldiag, xdiag, badj, col4, lane);
+      factor_piece4_mw(e, ldiag, xdiag, badj, stepA, stepX, warp, lane);
       if (lane == 0 && badj < 32) atomicMin(&bad, c0 + badj);
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        L[(c0 + lane) * LD + c0 + k] = (k < lane) ? e[k] : (k == lane ? ldiag : 0.f);
-        X[(c0 + k) * LD + c0 + lane] = (k > lane) ? e[k] : (k == lane ? xdiag : 0.f);
+      for (int q = 0; q < 8; ++q) {
+        const int k = 8 * warp + q;
+        L[(c0 + lane) * LD + c0 + k] = (k < lane) ? e[q] : (k == lane ? ldiag : 0.f);
+        X[(c0 + k) * LD + c0 + lane] = (k > lane) ? e[q] : (k == lane ? xdiag : 0.f);
       }
     } else {
-      // ---- inverse row blocks, alongside F (warps 1-15) ----
-      const int first = 32;
+      // ---- alongside F (warps 4-15): the previous piece's trailing update beyond the columns
+      // of this piece, then the inverse row blocks ----
+      const int first = 128;
+      if (kb >= 1) {
+        const int pc0 = c0 - 32, pnb4 = (NB - pc0 - 32) / 4;   // previous piece's trailing region
+        const int nrest = (pnb4 - 8) * (pnb4 - 7) / 2;        // lower tiles with bl >= 8
+        for (int t = tid - first; t < nrest; t += la::kInverseThreads) {
+          int bi, bl;
+          decode_tri(t, bi, bl);
+          trailing_tile(PT, L, pc0, bi + 8, bl + 8);
+        }
+      }
       if (kb >= 2) {
         inverse_row_product(X, OT + ((kb - 1) & 1) * 32 * LDT, kb - 1, first);
         named_barrier_or(la::kInverseBar, la::kInverseThreads, false);
@@ -434,30 +485,14 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
       }
     }
     __syncthreads();
-    // ---- T: A22 -= L21 L21^T (lower 4 x 4 tiles), and PT back into L's panel columns ----
+    // ---- T: A22 -= L21 L21^T on the next piece's 32 columns (lower 4 x 4 tiles with bl < 8),
+    // and PT back into L's panel columns; the tiles further right are left to warps 4-15 while
+    // the next piece is factored ----
     {
       const int nb4 = nbelow / 4;
-      const int nblk = nb4 * (nb4 + 1) / 2;
-      for (int blk = tid; blk < nblk; blk += 512) {
-        int bi, bl;
-        decode_tri(blk, bi, bl);
-        float acc[4][4] = {};
-#pragma unroll 8
-        for (int m = 0; m < 32; ++m) {
-          const float4 a4 = *reinterpret_cast<const float4*>(PT + m * LDT + 4 * bi);
-          const float4 b4 = *reinterpret_cast<const float4*>(PT + m * LDT + 4 * bl);
-          const float av[4] = {a4.x, a4.y, a4.z, a4.w}, bv[4] = {b4.x, b4.y, b4.z, b4.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-#pragma unroll
-            for (int v = 0; v < 4; ++v) acc[u][v] = fmaf(av[u], bv[v], acc[u][v]);
-        }
-        const int i0 = c0 + 32 + 4 * bi, l0 = c0 + 32 + 4 * bl;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            if (l0 + v <= i0 + u) L[(i0 + u) * LD + l0 + v] -= acc[u][v];
+      for (int it = tid; it < nb4 * 8; it += 512) {
+        const int bl = it & 7, bi = it >> 3;
+        if (bi >= bl) trailing_tile(PT, L, c0, bi, bl);
       }
       for (int e = tid; e < nbelow * 32; e += 512) {
         const int r = e >> 5, c = e & 31;
