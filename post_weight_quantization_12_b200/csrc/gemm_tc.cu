@@ -58,7 +58,6 @@ struct TcGemmParams {
   int stage_c;             // K <= 128 variant: C goes through shared memory by TMA
   int khi_from_m;
   int bstride;             // diagonal shift between batches (elements)
-  int split_ncols, split_row0;   // where the split output is written (K <= 128 variant)
 };
 
 // tile index -> (tm, tn): row-major over all tiles, or over the lower triangle tn <= tm
@@ -561,8 +560,7 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
             }
           }
           stop = !okc;
-          if (split && (p.split_ncols == 0 || n0 + 32 * j < p.split_ncols) &&
-              m0 + BM > p.split_row0) {
+          if (split) {
             // the tf32 split of the box, written row-contiguous from shared memory
             stop = named_barrier_or(kEpiBarrier, 128, stop || abort_flag);
             if (!stop) {
@@ -573,14 +571,12 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
                 const float4 v = *reinterpret_cast<const float4*>(
                     box + br * 128 + ((static_cast<uint32_t>(u) ^ static_cast<uint32_t>(br & 7)) << 4));
                 const int row = m0 + br, col = n0 + 32 * j + 4 * u;
-                if (row < p.M && row >= p.split_row0 &&
-                    (p.split_ncols == 0 || col < p.split_ncols)) {
+                if (row < p.M) {
                   const float4 bg = make_float4(tf32_round(v.x), tf32_round(v.y), tf32_round(v.z),
                                                 tf32_round(v.w));
                   const float4 sm = make_float4(v.x - bg.x, v.y - bg.y, v.z - bg.z, v.w - bg.w);
-                  const int64_t srow = row - p.split_row0;
-                  float* bp = p.Cbig + srow * p.ld_split + col;
-                  float* sp = p.Csmall + srow * p.ld_split + col;
+                  float* bp = p.Cbig + static_cast<int64_t>(row) * p.ld_split + col;
+                  float* sp = p.Csmall + static_cast<int64_t>(row) * p.ld_split + col;
                   if (col + 4 <= p.N) {
                     *reinterpret_cast<float4*>(bp) = bg;
                     *reinterpret_cast<float4*>(sp) = sm;
@@ -753,8 +749,6 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
   p.stage_c = 0;
   p.khi_from_m = g.khi_from_m;
   p.bstride = static_cast<int>(g.batch > 1 ? g.bstride : 0);
-  p.split_ncols = g.split_ncols;
-  p.split_row0 = g.split_row0;
   const bool panel = g.K > 0 && g.K <= tgp::kMaxK && !g.klo_from_m && !g.klo_from_n &&
                      !g.khi_from_m && g.batch == 1 && (!g.lower || g.M == g.N);
   if (panel) {
@@ -773,7 +767,6 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
     CUtensorMap tC;
     memset(&tC, 0, sizeof(tC));
     p.stage_c = (g.C != nullptr && p.vec4) ? 1 : 0;
-    if ((g.split_ncols != 0 || g.split_row0 != 0) && !p.stage_c) return GPTQ_EINVAL;
     if (p.stage_c &&
         (st = encode_tmap_2d(&tC, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, g.C, 4, g.N, g.M, g.ldc, 32,
                              tgp::BM, CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK)
@@ -782,7 +775,6 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
     const int smem = p.stage_c ? tgp::kSmemBytesStaged : tgp::kSmemBytes;
     gemm_tf32x3_panel_tc<<<grid, tgp::kThreads, smem, stream>>>(tAb, tAs, tBb, tBs, tC, p, g.info);
   } else {
-    if (g.split_ncols != 0 || g.split_row0 != 0) return GPTQ_EINVAL;
     const int64_t grid = static_cast<int64_t>(tiles_m) * p.tiles_n * g.batch;
     if (grid > 0x7fffffff) return GPTQ_EUNSUPPORTED;
     p.n_tiles = static_cast<int>(grid);

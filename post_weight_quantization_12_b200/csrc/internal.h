@@ -57,10 +57,6 @@ struct TcGemmArgs {
   int batch = 1;
   int64_t bstride = 0;
   int khi_from_m = 0;
-  // Restrict the split output to columns < split_ncols (0: all) and rows >= split_row0, written at
-  // row - split_row0. Only the K <= 128 product with C in shared memory supports a restriction.
-  int split_ncols = 0;
-  int split_row0 = 0;
 };
 gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream);
 

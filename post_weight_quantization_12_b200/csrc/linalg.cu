@@ -579,21 +579,17 @@ static gptq_status potrf_blocked(float* A, int64_t n, Split Lsp, Split Dsp, int6
     const int64_t m = n - k0 - nb;
     if (m == 0) break;
     float* A21 = A + (k0 + nb) * n + k0;
-    // the split of the panel comes from the previous trailing update's epilogue, except the first
-    if (k0 == 0) GPTQ_TRY(launch_split_tf32(A21, n, m, nb, Psp.b, Psp.s, kNB, stream));
+    GPTQ_TRY(launch_split_tf32(A21, n, m, nb, Psp.b, Psp.s, kNB, stream));
     // panel solve: L21 = A21 * Dinv^T, written to A and, split, to Lsp
     const int64_t loff = (k0 + nb) * n + k0;
     TcGemmArgs t{Psp.b, Psp.s, Dsp.b + doff, Dsp.s + doff, kNB, ld_dinv, 0, 0,
                  static_cast<int>(m), nb, nb, 1.f, 0.f, 0, 0, 0,
                  A21, n, Lsp.b + loff, Lsp.s + loff, n, info};
     GPTQ_TRY(launch_gemm_tc(t, stream));
-    // trailing update: A22 -= L21 L21^T (lower tiles); its epilogue also writes the tf32 split of
-    // the next panel (the first 128 columns below the next diagonal block) into Psp
+    // trailing update: A22 -= L21 L21^T (lower tiles)
     TcGemmArgs u{Lsp.b + loff, Lsp.s + loff, Lsp.b + loff, Lsp.s + loff, n, n, 0, 0,
                  static_cast<int>(m), static_cast<int>(m), nb, -1.f, 1.f, 1, 0, 0,
-                 A + (k0 + nb) * n + (k0 + nb), n, Psp.b, Psp.s, kNB, info};
-    u.split_ncols = kNB;
-    u.split_row0 = kNB;
+                 A + (k0 + nb) * n + (k0 + nb), n, nullptr, nullptr, 0, info};
     GPTQ_TRY(launch_gemm_tc(u, stream));
   }
   return GPTQ_OK;
