@@ -121,3 +121,19 @@ def test_gemm_lower_update_k128(n, K):
     below = tile[:, None] >= tile[None, :]
     assert np.all(C[~below] == C0[~below])
     _check(C, P, P, -1.0, 1.0, C0, mask=below)
+
+
+@pytest.mark.parametrize("M,N,K,b_mn,beta", [
+    (512, 768, 128, 1, 1.0),     # trailing-update shape: R slab MN-major, C read and written
+    (512, 640, 128, 0, 1.0),     # 640 columns: five 128-wide tile columns
+    (256, 256, 64, 1, 0.0),      # C written only
+    (1024, 384, 100, 0, 1.0),    # K not a multiple of the 32-wide stage
+])
+def test_gemm_k128_shapes(M, N, K, b_mn, beta):
+    """K <= 128 products at 256-multiple shapes: both B layouts, beta 0 and 1, ragged K."""
+    rng = np.random.default_rng(M + N + K + b_mn)
+    opA = rng.standard_normal((M, K)).astype(np.float32)
+    opBt = rng.standard_normal((N, K)).astype(np.float32)
+    C0 = rng.standard_normal((M, N)).astype(np.float32)
+    C, _, _ = _run(opA, 0, opBt, b_mn, alpha=-1.0, beta=beta, C0=C0)
+    _check(C, opA, opBt, -1.0, beta, C0)
