@@ -130,7 +130,7 @@ def test_gemm_lower_update_k128(n, K):
     (1024, 384, 100, 0, 1.0),    # K not a multiple of the 32-wide stage
 ])
 def test_gemm_k128_shapes(M, N, K, b_mn, beta):
-    """K <= 128 products at 256-multiple shapes: both B layouts, beta 0 and 1, ragged K."""
+    """K <= 128 products on multi-tile shapes: both B layouts, beta 0 and 1, ragged K."""
     rng = np.random.default_rng(M + N + K + b_mn)
     opA = rng.standard_normal((M, K)).astype(np.float32)
     opBt = rng.standard_normal((N, K)).astype(np.float32)
