@@ -58,11 +58,45 @@ class LayerQuantizer:
             return t.to(self.device, non_blocking=True)
         return t.to(self.device)
 
-    def add_batch(self, X: torch.Tensor):
-        """S += X^T X for token-major calibration inputs X [n_tokens, cols] (bf16 or fp32)."""
-        X = self._on_device(X)
-        _lib.hessian_accumulate(self.S, X, self.info, self.stream)
-        self.n_total += X.shape[0]
+    def add_batch(self, X: torch.Tensor, chunk_bytes: int = 256 << 20):
+        """S += X^T X for token-major calibration inputs X [n_tokens, cols] (bf16 or fp32).
+
+        A host tensor is copied in chunks of about `chunk_bytes` on a side stream into two device
+        buffers, so each chunk's copy overlaps the accumulation of the previous one."""
+        if X.device.type != "cpu":
+            X = self._on_device(X)
+            _lib.hessian_accumulate(self.S, X, self.info, self.stream)
+            self.n_total += X.shape[0]
+            return
+        if not X.is_pinned():
+            X = X.pin_memory()
+        n, cols = X.shape
+        rows_per = max(128, (chunk_bytes // max(1, cols * X.element_size())) // 128 * 128)
+        if n <= rows_per:
+            Xd = X.to(self.device, non_blocking=True)
+            _lib.hessian_accumulate(self.S, Xd, self.info, self.stream)
+            self.n_total += n
+            return
+        compute = self.stream if self.stream is not None else torch.cuda.current_stream(self.device)
+        copy = torch.cuda.Stream(self.device)
+        bufs = [torch.empty(rows_per, cols, dtype=X.dtype, device=self.device) for _ in range(2)]
+        free = [torch.cuda.Event(), torch.cuda.Event()]   # buffer b no longer read by S1
+        for b in range(2):
+            free[b].record(compute)
+        for i, r0 in enumerate(range(0, n, rows_per)):
+            b = i & 1
+            rows = min(rows_per, n - r0)
+            copy.wait_event(free[b])
+            with torch.cuda.stream(copy):
+                bufs[b][:rows].copy_(X[r0:r0 + rows], non_blocking=True)
+                landed = torch.cuda.Event()
+                landed.record(copy)
+            compute.wait_event(landed)
+            _lib.hessian_accumulate(self.S, bufs[b][:rows], self.info, compute)
+            free[b].record(compute)
+        self.n_total += n
+        for t in bufs:                     # keep the buffers alive until S1 has read them
+            t.record_stream(compute)
 
     def prepare(self):
         """H = 2S/N (kept in self.S) and R, the upper factor of (H + lambda I)^-1."""
@@ -93,8 +127,20 @@ class LayerQuantizer:
                          device=dev, dtype=torch.uint8)
         _lib.quantize_layer(W, self.R, bits, group, block, W_hat, codes, scales, zeros, err_sq, ws,
                             self.info, self.stream)
-        info = int(self.info.item())
         if to_host:
-            codes, scales, zeros, W_hat, err_sq = (t.cpu() for t in (codes, scales, zeros, W_hat,
-                                                                     err_sq))
+            # pinned host outputs, copied asynchronously on the same stream, one synchronization
+            stream = self.stream if self.stream is not None else torch.cuda.current_stream(dev)
+            outs = []
+            with torch.cuda.stream(stream):
+                for t in (codes, scales, zeros, W_hat, err_sq):
+                    h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+                    h.copy_(t, non_blocking=True)
+                    outs.append(h)
+                info_h = torch.empty(1, dtype=torch.int32, pin_memory=True)
+                info_h.copy_(self.info, non_blocking=True)
+            stream.synchronize()
+            codes, scales, zeros, W_hat, err_sq = outs
+            info = int(info_h.item())
+        else:
+            info = int(self.info.item())
         return QuantizedLayer(codes, scales, zeros, W_hat, err_sq, info)
