@@ -46,7 +46,8 @@ __device__ __forceinline__ void grid_params(float lo, float hi, float maxq, floa
 __device__ __forceinline__ float rint_quot(float w, float s, float inv_s) {
   const float y = w * inv_s;
   const float r = rintf(y);
-  if (0.5f - fabsf(y - r) > 1e-5f * fmaxf(1.f, fabsf(y))) return r;
+  // |y - r| < 0.5 - 1e-5 (|y| + 1): a margin at least as wide as 1e-5 max(1, |y|)
+  if (fabsf(y - r) < fmaf(-1e-5f, fabsf(y), 0.5f - 1e-5f)) return r;
   return rintf(__fdiv_rn(w, s));
 }
 
@@ -210,7 +211,7 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   auto colof = [&](int k) { return S * (k >> 2) + 4 * sub + (k & 3); };  // block column of v[k]
 
   float v[CPL];
-  uint8_t q8[CPL];
+  float qf[CPL];                  // codes of this lane's columns, converted when stored
   float err[CPL];
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
@@ -231,7 +232,7 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   }
 #pragma unroll
   for (int k = 0; k < CPL; ++k) {
-    q8[k] = 0;
+    qf[k] = 0.f;
     err[k] = 0.f;
   }
   const float maxq = static_cast<float>((1 << bits) - 1);
@@ -302,7 +303,7 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
           const float e = __fmul_rn(__fsub_rn(w, wh), inv_d[j]);
           e4[u] = e;
           v[4 * t + u] = own ? wh : v[4 * t + u];
-          q8[4 * t + u] = own ? static_cast<uint8_t>(q) : q8[4 * t + u];
+          qf[4 * t + u] = own ? q : qf[4 * t + u];
           err[4 * t + u] = own ? e : err[4 * t + u];
 #pragma unroll
           for (int u2 = u + 1; u2 < 4; ++u2) w4[u2] = fmaf(-e, Rz[j][j0 + u2], w4[u2]);
@@ -351,14 +352,14 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
       *reinterpret_cast<float4*>(eb) = make_float4(b4[0], b4[1], b4[2], b4[3]);
       *reinterpret_cast<float4*>(es) = make_float4(s4[0], s4[1], s4[2], s4[3]);
       *reinterpret_cast<uint32_t*>(cd) =
-          static_cast<uint32_t>(q8[4 * t]) | (static_cast<uint32_t>(q8[4 * t + 1]) << 8) |
-          (static_cast<uint32_t>(q8[4 * t + 2]) << 16) | (static_cast<uint32_t>(q8[4 * t + 3]) << 24);
+          static_cast<uint32_t>(qf[4 * t]) | (static_cast<uint32_t>(qf[4 * t + 1]) << 8) |
+          (static_cast<uint32_t>(qf[4 * t + 2]) << 16) | (static_cast<uint32_t>(qf[4 * t + 3]) << 24);
     } else {
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         if (c + u < nb) {
           wd[u] = v[4 * t + u];
-          cd[u] = q8[4 * t + u];
+          cd[u] = static_cast<uint8_t>(qf[4 * t + u]);
           eb[u] = b4[u];
           es[u] = s4[u];
         }
