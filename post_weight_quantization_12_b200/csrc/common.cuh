@@ -141,6 +141,17 @@ __device__ __forceinline__ bool named_barrier_or(uint32_t id, uint32_t nthreads,
   return r != 0;
 }
 
+// Programmatic dependent launch: kernels of this library are launched so that they may start
+// while the kernel before them in the stream finishes. griddep_wait() returns once that kernel
+// has completed and its memory is visible; every kernel calls it before its first global memory
+// access. griddep_launch_dependents() lets the next kernel be scheduled now (it still waits).
+__device__ __forceinline__ void griddep_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" :::);
+}
+
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }

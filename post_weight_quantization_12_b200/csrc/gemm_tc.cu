@@ -122,6 +122,8 @@ gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  griddep_wait();                       // the previous kernel's results are visible from here
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0 && nk > 0) {
@@ -357,6 +359,8 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_base_sh;
+  griddep_wait();                       // the previous kernel's results are visible from here
+  griddep_launch_dependents();
 
   if (warp == 0) {
     if (lane == 0) {
@@ -677,6 +681,9 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
 __global__ void split_tf32_kernel(const float* __restrict__ X, int64_t ldx, int64_t rows,
                                   int64_t cols, float* __restrict__ big, float* __restrict__ small,
                                   int64_t ldo) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   const int64_t total = rows * cols;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -693,9 +700,8 @@ gptq_status launch_split_tf32(const float* X, int64_t ldx, int64_t rows, int64_t
   if (rows <= 0 || cols <= 0) return GPTQ_OK;
   const int64_t total = rows * cols;
   const int grid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 16 * 148));
-  split_tf32_kernel<<<grid, 256, 0, stream>>>(X, ldx, rows, cols, big, small, ldo);
-  count_launch();
-  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+  return launch_pdl(split_tf32_kernel, dim3(grid), dim3(256), 0, stream, X, ldx, rows, cols, big,
+                    small, ldo);
 }
 
 static gptq_status operand_map(CUtensorMap* m, const float* base, int64_t ld, int mn_major,
@@ -773,16 +779,15 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
       return st;
     const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
     const int smem = p.stage_c ? tgp::kSmemBytesStaged : tgp::kSmemBytes;
-    gemm_tf32x3_panel_tc<<<grid, tgp::kThreads, smem, stream>>>(tAb, tAs, tBb, tBs, tC, p, g.info);
+    return launch_pdl(gemm_tf32x3_panel_tc, dim3(grid), dim3(tgp::kThreads), smem, stream, tAb,
+                      tAs, tBb, tBs, tC, p, g.info);
   } else {
     const int64_t grid = static_cast<int64_t>(tiles_m) * p.tiles_n * g.batch;
     if (grid > 0x7fffffff) return GPTQ_EUNSUPPORTED;
     p.n_tiles = static_cast<int>(grid);
-    gemm_tf32x3_tc<<<static_cast<unsigned>(grid), kThreads, kSmemBytes, stream>>>(tAb, tAs, tBb,
-                                                                                   tBs, p, g.info);
+    return launch_pdl(gemm_tf32x3_tc, dim3(static_cast<unsigned>(grid)), dim3(kThreads), kSmemBytes,
+                      stream, tAb, tAs, tBb, tBs, p, g.info);
   }
-  count_launch();
-  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }
 
 }  // namespace gptq

@@ -79,6 +79,27 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
 // Host-side count of kernels this library has enqueued (diagnostic, see gptq_kernel_launches).
 void count_launch(uint64_t n = 1);
 
+// Launch with programmatic stream serialization: the kernel may begin while the previous kernel
+// in the stream drains; it must call griddep_wait() before touching global memory. Counts the
+// launch and reports launch errors.
+template <typename... KArgs, typename... Args>
+inline gptq_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  count_launch();
+  return e == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+}
+
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 }  // namespace gptq

@@ -7,7 +7,7 @@
 //
 // Two routes to the same R (the upper factor with positive diagonal is unique):
 //  * three-step, as the pages write it: H_d = L L^T (blocked right-looking Cholesky, 128-wide
-//    panels), L^-1 (blocked triangular inverse, row block by row block), H_d^-1 = L^-T L^-1
+//    panels), L^-1 (triangular inverse by recursive doubling), H_d^-1 = L^-T L^-1
 //    (triangular product, lower half only), H_d^-1 = L2 L2^T (second Cholesky), R = L2^T;
 //  * reversed: with J the order-reversing permutation, J H_d J = M M^T (one Cholesky), so
 //    H_d = U U^T with U = J M J upper, H_d^-1 = U^-T U^-1 and R = U^-1 = J M^-1 J: one Cholesky
@@ -48,6 +48,9 @@ __device__ __forceinline__ float tf32_rna(float x) {
 __global__ void __launch_bounds__(1024)
 diag_lambda_kernel(const float* S, int64_t n, double scale, float damp_rel, float* lam_out,
                    int32_t* info) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   __shared__ double part[32];
   double s = 0.0;
   for (int64_t i = threadIdx.x; i < n; i += blockDim.x) s += static_cast<double>(S[i * n + i]);
@@ -76,6 +79,9 @@ __device__ __forceinline__ void decode_tri(int t, int& I, int& J) {
 // One 32 x 32 lower tile pair per CTA (blockDim 32 x 8).
 __global__ void __launch_bounds__(256)
 finalize_kernel(float* S_H, float* R, int64_t n, float scale, const float* lam_ptr) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   __shared__ float t[32][33];
   int I, J;
   decode_tri(blockIdx.x, I, J);
@@ -103,6 +109,9 @@ finalize_kernel(float* S_H, float* R, int64_t n, float scale, const float* lam_p
 
 // R = L2^T in place (L2 lower with zero upper): the result is upper with zero strict lower part.
 __global__ void __launch_bounds__(256) transpose_to_upper_kernel(float* R, int64_t n) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   __shared__ float t[32][33];
   int I, J;
   decode_tri(blockIdx.x, I, J);
@@ -130,6 +139,9 @@ __global__ void __launch_bounds__(256) transpose_to_upper_kernel(float* R, int64
 // J H_d J (entry [a][b] = H_d[n-1-a][n-1-b]) into R with its strict upper part zeroed.
 __global__ void __launch_bounds__(256)
 finalize_reversed_kernel(float* S_H, float* R, int64_t n, float scale, const float* lam_ptr) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   __shared__ float t[32][33];
   int I, J;
   decode_tri(blockIdx.x, I, J);
@@ -167,6 +179,9 @@ finalize_reversed_kernel(float* S_H, float* R, int64_t n, float scale, const flo
 // the result is upper, its strict lower part zeroed. One lower 32 x 32 tile of V per CTA.
 __global__ void __launch_bounds__(256)
 reverse_to_upper_kernel(float* R, const float* Vb, const float* Vs, int64_t n) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   int I, J;
   decode_tri(blockIdx.x, I, J);
   const int tx = threadIdx.x, ty = threadIdx.y;
@@ -375,6 +390,9 @@ __device__ __forceinline__ void trailing_tile(const float* PT, float* L, int c0,
 __global__ void __launch_bounds__(la::kDiagThreads)
 potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, int64_t ldd,
                   int32_t* info, int info_base, int rev_n, int store_l) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   constexpr int NB = 128, LD = la::kLd, LDT = la::kLdt;
   extern __shared__ float sm[];
   float* L = sm;
@@ -548,10 +566,8 @@ static gptq_status launch_potrf_diag(float* A, int64_t n, int k0, int nb, float*
       return GPTQ_ECUDA;
     attr_done = true;
   }
-  potrf_diag_kernel<<<1, la::kDiagThreads, la::kDiagSmem, stream>>>(A, n, k0, nb, Db, Ds, ldd, info,
-                                                                     info_base, rev_n, store_l);
-  count_launch();
-  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+  return launch_pdl(potrf_diag_kernel, dim3(1), dim3(la::kDiagThreads), la::kDiagSmem, stream, A, n,
+                    k0, nb, Db, Ds, ldd, info, info_base, rev_n, store_l ? 1 : 0);
 }
 
 struct Split {
@@ -673,19 +689,17 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
 
   // S2
   const double scale = 2.0 / static_cast<double>(n_total);
-  diag_lambda_kernel<<<1, 1024, 0, stream>>>(S_H, n, scale, damp_rel, w.lam, info);
-  count_launch();
-  if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
+  GPTQ_TRY(launch_pdl(diag_lambda_kernel, dim3(1), dim3(1024), 0, stream, S_H, n, scale, damp_rel,
+                      w.lam, info));
   const int nt = static_cast<int>((n + 31) / 32);
   const int ntri = nt * (nt + 1) / 2;
   const bool reversed = route != GPTQ_ROUTE_THREE_STEP;
   if (reversed)
-    finalize_reversed_kernel<<<ntri, dim3(32, 8), 0, stream>>>(S_H, R, n, static_cast<float>(scale),
-                                                               w.lam);
+    GPTQ_TRY(launch_pdl(finalize_reversed_kernel, dim3(ntri), dim3(32, 8), 0, stream, S_H, R, n,
+                        static_cast<float>(scale), w.lam));
   else
-    finalize_kernel<<<ntri, dim3(32, 8), 0, stream>>>(S_H, R, n, static_cast<float>(scale), w.lam);
-  count_launch();
-  if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
+    GPTQ_TRY(launch_pdl(finalize_kernel, dim3(ntri), dim3(32, 8), 0, stream, S_H, R, n,
+                        static_cast<float>(scale), w.lam));
 
   // S3: H_d = L L^T in R (reversed route: J H_d J = M M^T, M written as L below); the inverses of
   // L's diagonal blocks land in V (the split of L^-1)
@@ -697,9 +711,8 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
 
   if (reversed) {
     // R = J M^-1 J
-    reverse_to_upper_kernel<<<ntri, dim3(32, 8), 0, stream>>>(R, w.V.b, w.V.s, n);
-    count_launch();
-    return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+    return launch_pdl(reverse_to_upper_kernel, dim3(ntri), dim3(32, 8), 0, stream, R, w.V.b, w.V.s,
+                      n);
   }
 
   // S4b: H_d^-1 = L^-T L^-1 (lower tiles) into R
@@ -711,9 +724,7 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
   // S5: H_d^-1 = L2 L2^T (reusing the L split and the diagonal scratch), then R = L2^T
   GPTQ_TRY(potrf_blocked(R, n, w.L, w.D, kNB, false, w.P, info, static_cast<int>(n), 0, true,
                          stream));
-  transpose_to_upper_kernel<<<ntri, dim3(32, 8), 0, stream>>>(R, n);
-  count_launch();
-  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+  return launch_pdl(transpose_to_upper_kernel, dim3(ntri), dim3(32, 8), 0, stream, R, n);
 }
 
 }  // namespace gptq

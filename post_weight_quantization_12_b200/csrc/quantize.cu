@@ -22,6 +22,12 @@
 
 namespace gptq {
 
+#define GPTQ_TRY_Q(x)             \
+  do {                            \
+    gptq_status _s = (x);         \
+    if (_s != GPTQ_OK) return _s; \
+  } while (0)
+
 
 // tf32 rounding, for the (big, small) operand split of the trailing product
 __device__ __forceinline__ float tf32_rna_q(float x) {
@@ -63,6 +69,9 @@ __device__ __forceinline__ float load_w<__nv_bfloat16>(const __nv_bfloat16* p) {
 // bf16 rows of 8-element chunks (16-byte loads, two float4 stores); cols % 8 == 0, ldw % 8 == 0
 __global__ void convert_bf16_vec_kernel(const __nv_bfloat16* __restrict__ W, int64_t ldw,
                                         float* __restrict__ Wh, int64_t rows, int64_t cols) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   const int64_t c8 = cols / 8, total = rows * c8;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -80,6 +89,9 @@ __global__ void convert_bf16_vec_kernel(const __nv_bfloat16* __restrict__ W, int
 template <typename T>
 __global__ void convert_kernel(const T* __restrict__ W, int64_t ldw, float* __restrict__ Wh,
                                int64_t rows, int64_t cols) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   const int64_t total = rows * cols;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -91,6 +103,9 @@ __global__ void convert_kernel(const T* __restrict__ W, int64_t ldw, float* __re
 // One warp per row: grid of columns [c0, c0 + len) of the current weights.
 __global__ void params_kernel(const float* __restrict__ Wh, int64_t rows, int64_t cols, int64_t c0,
                               int64_t len, int bits, float* scales, uint8_t* zeros, int G, int gi) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   const int64_t row = blockIdx.x * static_cast<int64_t>(blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= rows) return;
@@ -128,6 +143,9 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
                    uint8_t* __restrict__ codes, float* __restrict__ Eb, float* __restrict__ Es,
                    float* __restrict__ err_sq, float* __restrict__ Rb_out,
                    float* __restrict__ Rs_out, int64_t nrest) {
+  griddep_wait();
+  griddep_launch_dependents();
+
   constexpr int S = 4 * TPR;       // columns covered by one float4 from each lane of a row
   constexpr int NT = B / S;        // float4 groups per lane
   constexpr int CPL = 4 * NT;      // columns per lane
@@ -396,11 +414,9 @@ static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, con
       return GPTQ_ECUDA;
     attr_done = true;
   }
-  column_loop_kernel<B, TPR, THREADS><<<static_cast<unsigned>(grid), THREADS, smem, stream>>>(
-      Wh, rows, cols, R, b0, nb, bits, group, group_mode, gi_fixed, scales, zeros, G, codes, Eb,
-      Es, err_sq, Rb, Rs, nrest);
-  count_launch();
-  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+  return launch_pdl(column_loop_kernel<B, TPR, THREADS>, dim3(static_cast<unsigned>(grid)),
+                    dim3(THREADS), smem, stream, Wh, rows, cols, R, b0, nb, bits, group, group_mode,
+                    gi_fixed, scales, zeros, G, codes, Eb, Es, err_sq, Rb, Rs, nrest);
 }
 
 gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, int64_t cols,
@@ -419,23 +435,23 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
   const int cgrid = static_cast<int>(std::min<int64_t>((total + 255) / 256, 8 * 148));
   if (w_dtype == GPTQ_BF16 && cols % 8 == 0 && ldw % 8 == 0 &&
       (reinterpret_cast<uintptr_t>(W) & 15) == 0)
-    convert_bf16_vec_kernel<<<std::min<int64_t>((total / 8 + 255) / 256, 8 * 148), 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(W), ldw, Wh, rows, cols);
+    GPTQ_TRY_Q(launch_pdl(convert_bf16_vec_kernel,
+                          dim3(static_cast<unsigned>(std::min<int64_t>((total / 8 + 255) / 256,
+                                                                       8 * 148))),
+                          dim3(256), 0, stream, static_cast<const __nv_bfloat16*>(W), ldw, Wh, rows,
+                          cols));
   else if (w_dtype == GPTQ_BF16)
-    convert_kernel<__nv_bfloat16><<<cgrid, 256, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(W), ldw, Wh, rows, cols);
+    GPTQ_TRY_Q(launch_pdl(convert_kernel<__nv_bfloat16>, dim3(cgrid), dim3(256), 0, stream,
+                          static_cast<const __nv_bfloat16*>(W), ldw, Wh, rows, cols));
   else
-    convert_kernel<float><<<cgrid, 256, 0, stream>>>(static_cast<const float*>(W), ldw, Wh, rows,
-                                                     cols);
-  count_launch();
-  if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
+    GPTQ_TRY_Q(launch_pdl(convert_kernel<float>, dim3(cgrid), dim3(256), 0, stream,
+                          static_cast<const float*>(W), ldw, Wh, rows, cols));
   if (err_sq != nullptr && cudaMemsetAsync(err_sq, 0, rows * sizeof(float), stream) != cudaSuccess)
     return GPTQ_ECUDA;
   const unsigned pgrid = static_cast<unsigned>((rows + 7) / 8);
   if (group <= 0) {
-    params_kernel<<<pgrid, 256, 0, stream>>>(Wh, rows, cols, 0, cols, bits, scales, zeros, 1, 0);
-    count_launch();
-    if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
+    GPTQ_TRY_Q(launch_pdl(params_kernel, dim3(pgrid), dim3(256), 0, stream, Wh, rows, cols, 0, cols,
+                          bits, scales, zeros, 1, 0));
   }
   for (int64_t b0 = 0; b0 < cols; b0 += block) {
     const int nb = static_cast<int>(cols - b0 < block ? cols - b0 : block);
@@ -444,10 +460,8 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
     if (group > 0 && group % block == 0 && group != block) {
       gi = static_cast<int>(b0 / group);
       if (b0 % group == 0) {
-        params_kernel<<<pgrid, 256, 0, stream>>>(Wh, rows, cols, b0, group, bits, scales, zeros, G,
-                                                 gi);
-        count_launch();
-        if (cudaGetLastError() != cudaSuccess) return GPTQ_ECUDA;
+        GPTQ_TRY_Q(launch_pdl(params_kernel, dim3(pgrid), dim3(256), 0, stream, Wh, rows, cols, b0,
+                              static_cast<int64_t>(group), bits, scales, zeros, G, gi));
       }
     } else if (group > 0) {
       mode = 1;

@@ -149,7 +149,8 @@ def test_prepare_reports_bad_hessian():
 # ------------------------------------------------------------------------------------------------
 
 @pytest.mark.parametrize("group,block", [(-1, 32), (-1, 128), (128, 128), (32, 128), (256, 128),
-                                         (64, 64), (16, 32)])
+                                         (64, 64), (16, 32), (8, 128), (4, 64), (2, 32),
+                                         (1, 32)])
 def test_identity_hessian_bit_exact_rtn(group, block):
     rows, cols, n = 96, 512, 1024
     W = synth.weights_np(synth.scaled_spec(synth.ATTN, rows, cols, 1), 3)
@@ -167,7 +168,7 @@ def test_identity_hessian_bit_exact_rtn(group, block):
 @pytest.mark.parametrize("rows,cols,bits,group,block", [
     (64, 128, 4, -1, 32), (200, 512, 4, 128, 128), (130, 512, 3, -1, 128),
     (64, 384, 4, 32, 64), (48, 1024, 4, 256, 128), (40, 200, 4, -1, 64), (64, 512, 2, 64, 32),
-    (33, 640, 8, 128, 128),
+    (33, 640, 8, 128, 128), (48, 256, 4, 8, 64), (40, 128, 4, 2, 32),
 ])
 def test_quantize_stagewise_against_oracle(rows, cols, bits, group, block):
     spec = synth.scaled_spec(synth.ATTN, rows, cols, 4 * cols)
