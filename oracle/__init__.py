@@ -4,3 +4,6 @@ from .gptq_oracle import (  # noqa: F401
     quantize, gptq_quantize, gptq_quantize_unbatched, rtn_quantize, layer_error, gptq_layer,
     check_shapes,
 )
+from .w4a16 import (  # noqa: F401
+    pack_codes, unpack_codes, dequantize, w4a16_matmul, w4a16_abs_terms, group_of_column,
+)
