@@ -55,6 +55,7 @@ def parse():
                         "then marked as not the configured workload)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-w4a16", action="store_true")
     p.add_argument("--cpu-sample-s", type=float, default=20.0)
     return p.parse_args()
 
@@ -252,6 +253,84 @@ def aggregate(elapsed_ms: float, launches: int, world: int, device):
     return float(t.item()), int(c.item())
 
 
+def bench_w4a16(dev, stream, peaks, peaks_src, iters=50):
+    """The W4A16 product on packed 4-bit codes (decode: one activation vector; and a batch of 8),
+    timed with CUDA events on the launching stream. Algorithmic bytes per launch: the packed codes
+    (rows * cols / 2), scales and zero points (5 bytes per row and group), the activations
+    (2 n cols) and the output (4 n rows). Inputs are larger than L2 (126 MB): the 12288 x 49152
+    layer holds 326 MB of weights, and the 4096 x 4096 case cycles through 24 separate layers."""
+    import torch
+    from post_weight_quantization_12_b200 import _lib, synth
+
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    info = torch.zeros(1, device=dev, dtype=torch.int32)
+
+    def make(rows, cols, group, seed):
+        codes, scales, zeros = synth.w4a16_operands_torch(rows, cols, group, seed, dev)
+        packed = torch.empty(rows, cols // 8, device=dev, dtype=torch.int32)
+        _lib.pack_codes_4bit(codes, packed, info, stream)
+        return codes, packed, scales, zeros
+
+    def timed(fn, reps):
+        for _ in range(3):
+            fn(0)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for k in range(reps):
+            fn(k)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps * 1e3          # us per launch
+
+    out = {"kernel": "w4a16_gemv_kernel", "bound": "hbm", "peak_gbs": hbm,
+           "peak_source": f"{peaks_src} HBM copy (kernel timed alone)", "cases": []}
+    cases = [("fc2_12288x49152_g128", 12288, 49152, 128, 1, 1),
+             ("fc2_12288x49152_g128", 12288, 49152, 128, 8, 1),
+             ("attn_4096x4096_g128 x24 layers", 4096, 4096, 128, 1, 24)]
+    made = {}
+    for name, rows, cols, group, n, layers in cases:
+        key = (rows, cols, group, layers)
+        if key not in made:
+            made.clear()
+            torch.cuda.empty_cache()
+            made[key] = [make(rows, cols, group, 100 + i) for i in range(layers)]
+        mats = made[key]
+        X = synth.inputs_torch(synth.scaled_spec(synth.ATTN, 1, cols, n), 7, dev)
+        Y = torch.empty(n, rows, device=dev)
+        G = cols // group
+
+        def fn(k, mats=mats, X=X, Y=Y, group=group):
+            _, packed, scales, zeros = mats[k % len(mats)]
+            _lib.w4a16_matmul(packed, scales, zeros, group, X, Y, info, stream)
+
+        us = timed(fn, max(iters, 2 * layers))
+        nbytes = rows * cols / 2 + 5.0 * rows * G + 2.0 * n * cols + 4.0 * n * rows
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out["cases"].append({"layer": name, "n": n, "us": us, "bytes": nbytes,
+                             "achieved_gbs": gbs, "frac": gbs / hbm,
+                             "weights_per_s": rows * cols / (us * 1e-6)})
+    # packing the quantizer's uint8 codes: reads rows * cols bytes, writes half of that
+    made.clear()
+    codes, packed, _, _ = make(12288, 49152, 128, 99)
+
+    def fp(k):
+        _lib.pack_codes_4bit(codes, packed, info, stream)
+
+    us = timed(fp, 20)
+    nbytes = 1.5 * codes.numel()
+    out["pack"] = {"kernel": "pack_codes_4bit_kernel", "layer": "12288x49152", "us": us,
+                   "bytes": nbytes, "achieved_gbs": nbytes / (us * 1e-6) / 1e9,
+                   "frac": nbytes / (us * 1e-6) / 1e9 / hbm}
+    torch.cuda.synchronize(dev)
+    if int(info.item()) != 0:
+        raise RuntimeError(f"device status {int(info.item())} in the W4A16 leg")
+    del codes, packed
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -411,6 +490,9 @@ def run_ours(args):
         raise RuntimeError(f"device status {int(info.item())} on the three-step route")
     line["S2_S5_routes_ms"] = {"reversed (default; the step above)": statistics.mean(s25),
                                "three_step": statistics.median(t3)}
+
+    if not args.no_w4a16:
+        line["w4a16"] = bench_w4a16(dev, stream, peaks, peaks_src)
 
     # end to end through the public API from pinned host buffers
     if not args.no_e2e:

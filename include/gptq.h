@@ -64,6 +64,7 @@ typedef enum gptq_route {
  *                   step route only). */
 #define GPTQ_INFO_TIMEOUT (-1)        /* a bounded wait inside a kernel expired */
 #define GPTQ_INFO_BAD_HESSIAN (-2)    /* mean(diag H) <= 0 or not finite: nothing to damp */
+#define GPTQ_INFO_BAD_CODE (-3)       /* gptq_pack_codes_4bit met a code >= 16 */
 
 /* Which workspace gptq_workspace_size() reports. */
 #define GPTQ_WS_PREPARE 1
@@ -209,6 +210,60 @@ gptq_status gptq_quantize_layer_noalloc(const void* W_dev, gptq_dtype w_dtype, i
                                         int group, int block, float* W_hat_dev, uint8_t* codes_dev,
                                         float* scales_dev, uint8_t* zeros_dev, float* err_sq_dev,
                                         int32_t* info_dev, void* stream);
+
+/*
+ * Packed 4-bit codes -- the storage the W4A16 product reads.
+ *
+ * Source: "GPTQ second-order quantization" blog, "What the original results established" (GPTQ
+ * is weight-only; the W4A16 runtime gains speed by moving fewer weight bytes and unpacking them
+ * in its kernel) and its Vietnamese version, "Group-wise quantization" (the packed layout is chosen
+ * together with the group size and the runtime kernel). The pages fix no layout; this one is:
+ *   eight codes per little-endian 32-bit word, row after row: code (r, c) is held in bits
+ *   4*(c % 8) .. 4*(c % 8) + 3 of word packed[r * (cols / 8) + c / 8]. Equivalently byte c / 2 of
+ *   row r holds column c in its low nibble when c is even and in its high nibble when c is odd.
+ *
+ *   codes_dev   uint8 [rows x ldc] (columns 0..cols-1 used), e.g. gptq_quantize_layer's codes at
+ *               bits <= 4. 8-byte aligned, ldc % 8 == 0.
+ *   packed_dev  uint32 [rows x cols/8], dense (row stride cols / 2 bytes), 4-byte aligned; written.
+ *   info_dev    status word (may be NULL): GPTQ_INFO_BAD_CODE if a code is 16 or more; its low
+ *               four bits are stored.
+ * rows == 0 enqueues nothing. Errors: GPTQ_EINVAL (null pointers, cols <= 0, cols % 8 != 0,
+ * ldc < cols, alignment).
+ */
+gptq_status gptq_pack_codes_4bit(const uint8_t* codes_dev, int64_t rows, int64_t cols, int64_t ldc,
+                                 uint32_t* packed_dev, int32_t* info_dev, void* stream);
+
+/*
+ * W4A16 product: Y = X W_hat^T with W_hat read from packed 4-bit codes and dequantized on the fly,
+ *   Y[n][r] = sum_c X[n][c] * s[r, g(c)] * (q[r][c] - z[r, g(c)]),  g(c) = c / group (0 per row).
+ *
+ * Source: "GPTQ second-order quantization" blog, "What the original results established" (W4A16:
+ * BF16 activations, weight bytes moved packed and dequantized in the kernel) and "Group-wise
+ * quantization" (scale and zero point per row or per group of input channels). One call serves a
+ * decode step (n = 1, a matrix-vector product) or a small batch of activation vectors (n <= 16).
+ *
+ *   packed_dev  codes in the layout of gptq_pack_codes_4bit, [rows x cols/8] uint32, 16-byte
+ *               aligned.
+ *   scales_dev  float32 [rows x G], zeros_dev uint8 [rows x G] (as gptq_quantize_layer writes
+ *               them); G = 1 for group == -1, else cols / group. Zero points above 127 are not
+ *               supported (4-bit quantizers produce 0..15).
+ *   group       -1 (per row) or a multiple of 128 that divides cols.
+ *   X_dev       activations [n x ldx], token-major, x_dtype GPTQ_BF16 only; 16-byte aligned,
+ *               ldx % 8 == 0, ldx >= cols.
+ *   Y_dev       float32 [n x ldy] output, ldy >= rows; fully overwritten in columns 0..rows-1.
+ *   info_dev    status word (may be NULL): GPTQ_INFO_TIMEOUT if a copy wait expires.
+ * Empty calls (rows == 0 or n == 0) are checked for shapes only and may pass NULL buffers.
+ * Arithmetic: q - z is formed exactly in bf16 and multiplied by X on the tensor cores with fp32
+ * accumulation over each 128-column chunk; the chunk sum is scaled by s in fp32 and the chunks
+ * are added in a fixed order, so results are deterministic for a given device and shape.
+ * rows == 0 or n == 0 enqueues nothing. Errors: GPTQ_EINVAL (null pointers, cols <= 0,
+ * cols % 32 != 0, group rules, ld or alignment rules, n < 0), GPTQ_EUNSUPPORTED (x_dtype other than
+ * GPTQ_BF16, n > 16, rows above 2^27, cols above 2^22).
+ */
+gptq_status gptq_w4a16_matmul(const uint32_t* packed_dev, const float* scales_dev,
+                              const uint8_t* zeros_dev, int64_t rows, int64_t cols, int group,
+                              const void* X_dev, gptq_dtype x_dtype, int64_t n, int64_t ldx,
+                              float* Y_dev, int64_t ldy, int32_t* info_dev, void* stream);
 
 /* Workspace bytes needed by one call (GPTQ_WS_PREPARE or GPTQ_WS_QUANTIZE); 0 for bad input. */
 size_t gptq_workspace_size(int which, int64_t rows, int64_t cols, int block);

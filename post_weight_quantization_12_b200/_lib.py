@@ -17,6 +17,7 @@ GPTQ_OK, GPTQ_EINVAL, GPTQ_ENOTPD, GPTQ_ECUDA, GPTQ_EUNSUPPORTED, GPTQ_ETIMEOUT,
 GPTQ_BF16, GPTQ_FP32 = 0, 1
 GPTQ_INFO_TIMEOUT = -1
 GPTQ_INFO_BAD_HESSIAN = -2
+GPTQ_INFO_BAD_CODE = -3
 GPTQ_WS_PREPARE, GPTQ_WS_QUANTIZE = 1, 2
 GPTQ_ROUTE_DEFAULT, GPTQ_ROUTE_THREE_STEP, GPTQ_ROUTE_REVERSED = 0, 1, 2
 GPTQ_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
@@ -36,6 +37,9 @@ SIGNATURES = {
     "gptq_quantize_layer_noalloc": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _I32, _I32, _I32, _P,
                                            _P, _P, _P, _P, _P, _P]),
     "gptq_kernel_launches": (ctypes.c_uint64, []),
+    "gptq_pack_codes_4bit": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "gptq_w4a16_matmul": (_I32, [_P, _P, _P, _I64, _I64, _I32, _P, _I32, _I64, _I64, _P, _I64, _P,
+                                 _P]),
     "gptq_selftest_gemm": (_I32, [_P, _I64, _I32, _P, _I64, _I32, _P, _I64, _I32, _I32, _I32,
                                   _F, _F, _I32, _I32, _I32, _P, _P, _P, _SZ, _P, _P]),
     "gptq_selftest_wait_timeout": (_I32, [_P, _I32, _P]),
@@ -165,6 +169,30 @@ def quantize_layer_noalloc(W, R, bits, group, block, W_hat, codes, scales, zeros
         int(block), _ptr(W_hat), _ptr(codes), _ptr(scales), _ptr(zeros), _ptr(err_sq), _ptr(info),
         _stream(stream))
     _check(st, "gptq_quantize_layer_noalloc")
+
+
+def pack_codes_4bit(codes, packed, info=None, stream=None):
+    """uint8 codes[rows, >= cols] -> packed[rows, cols // 8] (int32 or uint32 tensor, the 32-bit
+    words of the layout in include/gptq.h); cols = 8 * packed.shape[1]."""
+    ldc = _row_major_ld(codes, "codes")
+    if packed.dim() != 2 or not packed.is_contiguous() or packed.element_size() != 4:
+        raise ValueError("packed must be a contiguous 2-D tensor of 32-bit words")
+    st = load().gptq_pack_codes_4bit(_ptr(codes), codes.shape[0], 8 * packed.shape[1], ldc,
+                                     _ptr(packed), _ptr(info), _stream(stream))
+    _check(st, "gptq_pack_codes_4bit")
+
+
+def w4a16_matmul(packed, scales, zeros, group, X, Y, info=None, stream=None):
+    """Y[n, rows] (fp32) = X[n, cols] (bf16) @ W_hat^T with W_hat dequantized from the packed
+    4-bit codes[rows, cols // 8] and the scales / zeros [rows, G]."""
+    if packed.dim() != 2 or not packed.is_contiguous() or packed.element_size() != 4:
+        raise ValueError("packed must be a contiguous 2-D tensor of 32-bit words")
+    ldx = _row_major_ld(X, "X")
+    ldy = _row_major_ld(Y, "Y")
+    st = load().gptq_w4a16_matmul(_ptr(packed), _ptr(scales), _ptr(zeros), packed.shape[0],
+                                  8 * packed.shape[1], int(group), _ptr(X), _dtype_code(X),
+                                  X.shape[0], ldx, _ptr(Y), ldy, _ptr(info), _stream(stream))
+    _check(st, "gptq_w4a16_matmul")
 
 
 def selftest_gemm(A, a_mn, B, b_mn, C, M, N, K, alpha=1.0, beta=0.0, lower=False,

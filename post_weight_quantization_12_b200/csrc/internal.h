@@ -76,6 +76,13 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
                                float* W_hat, uint8_t* codes, float* scales, uint8_t* zeros,
                                float* err_sq, void* ws, int32_t* info, cudaStream_t stream);
 
+// Packed 4-bit codes and the W4A16 product (w4a16.cu).
+gptq_status run_pack_codes_4bit(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ldc,
+                                uint32_t* packed, int32_t* info, cudaStream_t stream);
+gptq_status run_w4a16_gemv(const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                           int64_t rows, int64_t cols, int group, const void* x, int64_t n,
+                           int64_t ldx, float* y, int64_t ldy, int32_t* info, cudaStream_t stream);
+
 // Host-side count of kernels this library has enqueued (diagnostic, see gptq_kernel_launches).
 void count_launch(uint64_t n = 1);
 

@@ -1,0 +1,396 @@
+// Packed 4-bit weights and the W4A16 product that consumes them.
+//
+// "GPTQ second-order quantization" blog, "What the original results established": GPTQ is
+// weight-only; in the W4A16 path the activations stay BF16 and the speed comes from moving fewer
+// weight bytes through a kernel that unpacks and dequantizes them ("Group-wise quantization": one
+// scale and zero point per row or per group of input channels, with the group size traded against
+// scale traffic). The product is HBM-bound: every weight code is read once, so the kernel is built
+// around keeping enough code bytes in flight (a TMA ring per warp) and spending as few
+// instructions per weight as possible (two-code-at-a-time dequantization, tensor-core dot
+// products).
+//
+// Layout of the packed codes: eight codes per little-endian 32-bit word, row after row; code
+// (r, c) sits in bits 4 (c mod 8) .. 4 (c mod 8) + 3 of word (r, c div 8).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace gptq {
+namespace {
+
+// ------------------------------------------------------------------------------------------------
+// Packing
+// ------------------------------------------------------------------------------------------------
+
+// One thread per output word: eight consecutive codes of a row (8 bytes) -> one 32-bit word.
+__global__ void __launch_bounds__(256)
+pack_codes_4bit_kernel(const uint8_t* __restrict__ codes, int64_t rows, int64_t words_per_row,
+                       int64_t ldc, uint32_t* __restrict__ packed, int32_t* info) {
+  griddep_wait();
+  const int64_t total = rows * words_per_row;
+  bool bad = false;
+  for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < total;
+       k += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = k / words_per_row, w = k - r * words_per_row;
+    const uint2 v = __ldg(reinterpret_cast<const uint2*>(codes + r * ldc + 8 * w));
+    bad |= ((v.x | v.y) & 0xF0F0F0F0u) != 0u;
+    // Bytes of v.x are codes 8w .. 8w+3, of v.y codes 8w+4 .. 8w+7. Word byte i must hold codes
+    // 2i (low nibble) and 2i+1 (high nibble).
+    const uint32_t a = v.x & 0x0F0F0F0Fu, b = v.y & 0x0F0F0F0Fu;
+    const uint32_t even = __byte_perm(a, b, 0x6420);  // codes 0, 2, 4, 6
+    const uint32_t odd = __byte_perm(a, b, 0x7531);   // codes 1, 3, 5, 7
+    packed[k] = even | (odd << 4);
+  }
+  if (bad) record_info(info, GPTQ_INFO_BAD_CODE);
+  griddep_launch_dependents();
+}
+
+// ------------------------------------------------------------------------------------------------
+// W4A16 product
+// ------------------------------------------------------------------------------------------------
+constexpr int kMt = 16;                          // rows of one mma tile (the mma's M)
+constexpr int kRows = 32;                        // rows of one CTA: two mma tiles per warp
+constexpr int kChunk = 128;                      // columns a warp takes per step: 4 lanes x 32
+constexpr int kStages = 3;                       // TMA ring depth per warp
+constexpr int kStageBytes = kRows * kChunk / 2;  // 32 rows x 64 bytes of codes
+constexpr int kMaxWarps = 16;
+
+// D = A * B + C for one m16n8k16 tile, bf16 inputs, fp32 accumulation.
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// d = a * b + c on bf16 pairs (one packed half-precision FMA instruction).
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// The eight codes of one word as four bf16 pairs (q_p - z, q_{p+4} - z), p = 0..3. The nibbles
+// are first split into bytes (even nibbles of w in `lo`, odd ones in `hi`); a byte permute then
+// pairs two of those bytes with the byte 0x43 above each, making two bf16 numbers whose exponent
+// is 2^7 and whose unit in the last place is 1, i.e. exactly 128 + q. Adding -(128 + z) (`negz`,
+// both halves) is exact too (integers of magnitude below 256), so the tensor core sees the exact
+// q - z. (A byte permute plus masks measured faster here than shift-and-mask extraction.)
+__device__ __forceinline__ void dequant_word(uint32_t w, uint32_t negz, uint32_t (&p)[4]) {
+  constexpr uint32_t kOne = 0x3F803F80u;    // (1.0, 1.0) in bf16
+  constexpr uint32_t kMagic = 0x43434343u;  // high byte of bf16 128.0, in every byte
+  const uint32_t lo = w & 0x0F0F0F0Fu;         // bytes: q0 q2 q4 q6
+  const uint32_t hi = (w >> 4) & 0x0F0F0F0Fu;  // bytes: q1 q3 q5 q7
+  p[0] = bf16x2_fma(__byte_perm(lo, kMagic, 0x4240), kOne, negz);  // (q0, q4)
+  p[1] = bf16x2_fma(__byte_perm(hi, kMagic, 0x4240), kOne, negz);  // (q1, q5)
+  p[2] = bf16x2_fma(__byte_perm(lo, kMagic, 0x4341), kOne, negz);  // (q2, q6)
+  p[3] = bf16x2_fma(__byte_perm(hi, kMagic, 0x4341), kOne, negz);  // (q3, q7)
+}
+
+// y[n][r] = sum_c x[n][c] * s[r, g(c)] * (q[r][c] - z[r, g(c)]) for 32 rows per CTA. Each of
+// the CTA's W warps takes the 128-column chunks w, w + W, w + 2W, ... and streams their codes
+// through its own ring of kStages TMA buffers (one 32 x 128 tile each); the warps' partial sums
+// are added in warp order at the end, so the result does not depend on timing.
+//
+// Per chunk and warp, lane (g = lane / 4, t = lane % 4) holds 32 codes (columns 32t .. 32t + 31
+// of the chunk) of each of the rows g, g + 8 (mma tile 0) and g + 16, g + 24 (mma tile 1), and
+// the activations of vector n = g (NT = 2: also n = g + 8); both tiles use the same activation
+// fragments. The mma's k index is a permutation of the columns, the same for both operands: in
+// step 2i (2i + 1) lane t's k slots {2t, 2t+1, 2t+8, 2t+9} are its columns 8i + {0, 4, 1, 5}
+// ({2, 6, 3, 7}), which is the order the nibble pairs come out of dequant_word.
+// Eight steps cover the chunk; its sum is then scaled by the row's group scale in fp32.
+// The group of chunk ch is (ch * gmul) >> 32 with gmul = ceil(2^32 / (group / 128)) -- exact for
+// the sizes the host admits -- and gmul = 0 for one scale per row.
+// Activation rows n >= n_act read row n_act - 1 (their products land in output columns that are
+// never stored); columns past `cols` (a ragged last chunk) read zeros.
+template <int NT>
+__global__ void __launch_bounds__(kMaxWarps * 32) __maxnreg__(NT == 1 ? 72 : 128)
+w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const float* __restrict__ scales,
+                  const uint8_t* __restrict__ zeros, int rows, int cols, uint64_t gmul,
+                  int n_groups, const __nv_bfloat16* __restrict__ x, int n_act, int64_t ldx,
+                  float* __restrict__ y, int64_t ldy, int32_t* info) {
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ volatile int abort_flag;
+  const int nwarps = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  uint8_t* ring = smem + warp * (kStages * kStageBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + nwarps * (kStages * kStageBytes)) +
+                   warp * kStages;
+  const int row0 = blockIdx.x * kRows;
+  const int nchunks = (cols + kChunk - 1) / kChunk;
+  const int full_chunks = cols / kChunk;
+
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    fence_mbarrier_init();
+  }
+  if (threadIdx.x == 0) abort_flag = 0;
+  __syncthreads();
+  griddep_wait();
+
+  int issued = 0;  // loads this warp has started (lane 0's count)
+  if (lane == 0) {
+    prefetch_tmap(&tcodes);
+    for (int s = 0; s < kStages; ++s) {
+      const int ch = warp + s * nwarps;
+      if (ch >= nchunks) break;
+      mbar_arrive_expect_tx(&bars[s], kStageBytes);
+      tma_load_2d(ring + s * kStageBytes, &tcodes, &bars[s], ch * (kChunk / 8), row0);
+      ++issued;
+    }
+  }
+
+  // Rows past the end read the last row's metadata (their results are not stored).
+  const float* srow[4];
+  const uint8_t* zrow[4];
+#pragma unroll
+  for (int m = 0; m < 4; ++m) {
+    const int r = min(row0 + g + 8 * m, rows - 1);
+    srow[m] = scales + static_cast<int64_t>(r) * n_groups;
+    zrow[m] = zeros + static_cast<int64_t>(r) * n_groups;
+  }
+  const __nv_bfloat16* xl[NT];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt)
+    xl[nt] = x + static_cast<int64_t>(min(nt * 8 + g, n_act - 1)) * ldx + 32 * t;
+
+  float acc[2][NT][4];
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[h][nt][e] = 0.f;
+
+  bool ok = true;
+  int j = 0;  // chunks this warp has consumed
+  uint32_t phase = 0;
+  for (int base = warp; ok && base < nchunks; base += kStages * nwarps, phase ^= 1u) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) {
+      const int ch = base + s * nwarps;
+      if (ch >= nchunks) break;
+      const uint32_t gi = static_cast<uint32_t>((static_cast<uint64_t>(ch) * gmul) >> 32);
+      float sc[4];
+      uint32_t nz[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        sc[m] = __ldg(srow[m] + gi);
+        nz[m] = (0xC300u + __ldg(zrow[m] + gi)) * 0x00010001u;  // -(128 + z), twice
+      }
+      uint4 xv[NT][4];
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const uint4* xp = reinterpret_cast<const uint4*>(xl[nt] + ch * kChunk);
+        if (ch < full_chunks) {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xv[nt][i] = __ldg(xp + i);
+        } else {
+          const bool in_cols = ch * kChunk + 32 * t < cols;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xv[nt][i] = in_cols ? __ldg(xp + i) : make_uint4(0, 0, 0, 0);
+        }
+      }
+
+      const bool got = __all_sync(0xffffffffu,
+                                  mbar_wait_bounded(&bars[s], phase, &abort_flag, info));
+      if (!got) {
+        ok = false;
+        break;
+      }
+      const uint8_t* st = ring + s * kStageBytes + g * 64 + t * 16;
+      uint4 wv[4];
+#pragma unroll
+      for (int m = 0; m < 4; ++m) wv[m] = *reinterpret_cast<const uint4*>(st + m * 8 * 64);
+
+      float d[2][NT][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d[h][nt][e] = 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint32_t b[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          const uint4 v = xv[nt][i];  // x[8i .. 8i+7] of this lane's columns, natural order
+          b[nt][0] = __byte_perm(v.x, v.z, 0x5410);  // (x0, x4)
+          b[nt][1] = __byte_perm(v.x, v.z, 0x7632);  // (x1, x5)
+          b[nt][2] = __byte_perm(v.y, v.w, 0x5410);  // (x2, x6)
+          b[nt][3] = __byte_perm(v.y, v.w, 0x7632);  // (x3, x7)
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t w_lo = i == 0 ? wv[2 * h].x : i == 1 ? wv[2 * h].y
+                              : i == 2 ? wv[2 * h].z : wv[2 * h].w;
+          const uint32_t w_hi = i == 0 ? wv[2 * h + 1].x : i == 1 ? wv[2 * h + 1].y
+                              : i == 2 ? wv[2 * h + 1].z : wv[2 * h + 1].w;
+          uint32_t p0[4], p1[4];
+          dequant_word(w_lo, nz[2 * h], p0);
+          dequant_word(w_hi, nz[2 * h + 1], p1);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt) {
+            mma_bf16(d[h][nt], p0[0], p1[0], p0[1], p1[1], b[nt][0], b[nt][1]);
+            mma_bf16(d[h][nt], p0[2], p1[2], p0[3], p1[3], b[nt][2], b[nt][3]);
+          }
+        }
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          acc[h][nt][0] = fmaf(sc[2 * h], d[h][nt][0], acc[h][nt][0]);
+          acc[h][nt][1] = fmaf(sc[2 * h], d[h][nt][1], acc[h][nt][1]);
+          acc[h][nt][2] = fmaf(sc[2 * h + 1], d[h][nt][2], acc[h][nt][2]);
+          acc[h][nt][3] = fmaf(sc[2 * h + 1], d[h][nt][3], acc[h][nt][3]);
+        }
+      ++j;
+
+      // Every lane has consumed stage s (its codes fed the products above): refill it.
+      __syncwarp();
+      if (lane == 0) {
+        const int nxt = ch + kStages * nwarps;
+        if (nxt < nchunks) {
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&bars[s], kStageBytes);
+          tma_load_2d(ring + s * kStageBytes, &tcodes, &bars[s], nxt * (kChunk / 8), row0);
+          ++issued;
+        }
+      }
+    }
+  }
+  griddep_launch_dependents();
+
+  if (!ok && lane == 0) {
+    // Let the loads still in flight land before the ring is reused or the CTA exits.
+    for (int k = j; k < issued; ++k) mbar_drain_bounded(&bars[k % kStages], (k / kStages) & 1);
+  }
+  __syncwarp();
+
+  // Partial sums of this warp -> its (now idle) ring: part[row][n], 32 x 8NT floats.
+  float* part = reinterpret_cast<float*>(ring);
+  constexpr int kLd = 8 * NT;
+#pragma unroll
+  for (int h = 0; h < 2; ++h)
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int ra = h * kMt + g, rb = h * kMt + g + 8;
+      part[ra * kLd + nt * 8 + 2 * t] = acc[h][nt][0];
+      part[ra * kLd + nt * 8 + 2 * t + 1] = acc[h][nt][1];
+      part[rb * kLd + nt * 8 + 2 * t] = acc[h][nt][2];
+      part[rb * kLd + nt * 8 + 2 * t + 1] = acc[h][nt][3];
+    }
+  __syncthreads();
+  if (abort_flag) return;
+  for (int k = threadIdx.x; k < kRows * kLd; k += blockDim.x) {
+    const int row = k % kRows, n = k / kRows;
+    const int r = row0 + row;
+    if (n >= n_act || r >= rows) continue;
+    float sum = 0.f;
+    for (int w = 0; w < nwarps; ++w)
+      sum += reinterpret_cast<const float*>(smem + w * (kStages * kStageBytes))[row * kLd + n];
+    y[static_cast<int64_t>(n) * ldy + r] = sum;
+  }
+}
+
+size_t gemv_smem_bytes(int nwarps) {
+  return static_cast<size_t>(nwarps) * kStages * (kStageBytes + 8);
+}
+
+// Warps per CTA for a layer of `ctas` CTAs: the most warps per CTA whose CTAs all fit on the
+// device at once (no second, partial wave of CTAs at the end); if no choice fits them all, the one
+// with the most warps resident. Occupancy per warp count comes from the runtime (registers and
+// shared memory of the kernel as built) and is cached per device.
+template <int NT>
+int pick_warps(int64_t ctas, int64_t nchunks) {
+  static int occ[64][kMaxWarps + 1] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
+  if (occ[dev][0] == 0) {
+    if (cudaFuncSetAttribute(w4a16_gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(gemv_smem_bytes(kMaxWarps))) != cudaSuccess)
+      return -1;
+    for (int w = 1; w <= kMaxWarps; ++w) {
+      int b = 0;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, w4a16_gemv_kernel<NT>, 32 * w,
+                                                        gemv_smem_bytes(w)) != cudaSuccess)
+        return -1;
+      occ[dev][w] = b;
+    }
+    occ[dev][0] = 1;
+  }
+  const int64_t sms = num_sms();
+  int best = 1;
+  int64_t best_resident = -1;
+  bool best_fits = false;
+  for (int w = 1; w <= kMaxWarps && w <= nchunks; ++w) {
+    const int64_t slots = static_cast<int64_t>(occ[dev][w]) * sms;
+    if (slots <= 0) continue;
+    const bool fits = ctas <= slots;
+    const int64_t resident = (fits ? ctas : slots) * w;
+    if ((fits && !best_fits) || (fits == best_fits && resident > best_resident)) {
+      best = w;
+      best_resident = resident;
+      best_fits = fits;
+    }
+  }
+  return best;
+}
+
+template <int NT>
+gptq_status launch_gemv(const CUtensorMap& tmap, int64_t rows, int64_t cols, const float* scales,
+                        const uint8_t* zeros, uint64_t gmul, int n_groups,
+                        const __nv_bfloat16* x, int n, int64_t ldx, float* y, int64_t ldy,
+                        int32_t* info, cudaStream_t stream) {
+  const int64_t ctas = (rows + kRows - 1) / kRows;
+  const int nwarps = pick_warps<NT>(ctas, (cols + kChunk - 1) / kChunk);
+  if (nwarps <= 0) return GPTQ_ECUDA;
+  return launch_pdl(w4a16_gemv_kernel<NT>, dim3(static_cast<unsigned>(ctas)), dim3(nwarps * 32),
+                    gemv_smem_bytes(nwarps), stream, tmap, scales, zeros, static_cast<int>(rows),
+                    static_cast<int>(cols), gmul, n_groups, x, n, ldx, y, ldy, info);
+}
+
+}  // namespace
+
+gptq_status run_pack_codes_4bit(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ldc,
+                                uint32_t* packed, int32_t* info, cudaStream_t stream) {
+  const int64_t words = rows * (cols / 8);
+  int64_t blocks = (words + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  return launch_pdl(pack_codes_4bit_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                    stream, codes, rows, cols / 8, ldc, packed, info);
+}
+
+gptq_status run_w4a16_gemv(const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                           int64_t rows, int64_t cols, int group, const void* x, int64_t n,
+                           int64_t ldx, float* y, int64_t ldy, int32_t* info,
+                           cudaStream_t stream) {
+  CUtensorMap tmap;
+  gptq_status st = encode_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, 4, cols / 8,
+                                  rows, cols / 8, kChunk / 8, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != GPTQ_OK) return st;
+  const int n_groups = group > 0 ? static_cast<int>(cols / group) : 1;
+  // chunk -> group index as (chunk * gmul) >> 32 with gmul = ceil(2^32 / d), d = group / 128
+  // chunks per group: exact while chunk * d <= 2^32, which cols <= 2^22 guarantees. gmul = 0
+  // maps every chunk to group 0 (one scale per row).
+  const uint64_t d = group > 0 ? static_cast<uint64_t>(group / kChunk) : 0;
+  const uint64_t gmul = d == 0 ? 0 : ((1ull << 32) + d - 1) / d;
+  const auto* xb = static_cast<const __nv_bfloat16*>(x);
+  if (n <= 8)
+    return launch_gemv<1>(tmap, rows, cols, scales, zeros, gmul, n_groups, xb,
+                          static_cast<int>(n), ldx, y, ldy, info, stream);
+  return launch_gemv<2>(tmap, rows, cols, scales, zeros, gmul, n_groups, xb, static_cast<int>(n),
+                        ldx, y, ldy, info, stream);
+}
+
+}  // namespace gptq

@@ -172,3 +172,28 @@ def inputs_torch(spec: LayerSpec, seed: int, device, n_tokens: int | None = None
             v = z * torch.rsqrt(c / 3.0) * scale
         x[t0:t1] = v.to(dt)
     return x
+
+
+# ----------------------------------------------------------------------------------------------
+# Quantized-weight operands for the W4A16 product
+# ----------------------------------------------------------------------------------------------
+
+def w4a16_operands_torch(rows: int, cols: int, group: int, seed: int, device="cpu"):
+    """Stand-in quantized layer for timing and parity of the W4A16 product, drawn on ``device``:
+    codes uint8 [rows, cols] uniform in 0..15 (seed+0); scales float32 [rows, G] log-uniform in
+    [1e-3, 1e-2] (the step of a 4-bit grid over weights of std 0.01-0.02) and zero points uint8
+    [rows, G] uniform in 0..15 (seed+1); G = 1 for group <= 0, else cols // group."""
+    import torch
+    G = 1 if group <= 0 else cols // group
+    gc = torch.Generator(device=device).manual_seed(seed + 0)
+    gm = torch.Generator(device=device).manual_seed(seed + 1)
+    codes = torch.empty(rows, cols, dtype=torch.uint8, device=device)
+    chunk = max(1, (1 << 26) // max(cols, 1))
+    for r0 in range(0, rows, chunk):
+        r1 = min(rows, r0 + chunk)
+        codes[r0:r1] = torch.randint(0, 16, (r1 - r0, cols), generator=gc, device=device,
+                                     dtype=torch.uint8)
+    scales = torch.exp(torch.empty(rows, G, device=device).uniform_(
+        math.log(1e-3), math.log(1e-2), generator=gm))
+    zeros = torch.randint(0, 16, (rows, G), generator=gm, device=device, dtype=torch.uint8)
+    return codes, scales, zeros

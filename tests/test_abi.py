@@ -88,3 +88,35 @@ def test_other_entry_points_reject_bad_arguments(built_lib):
                                  FAKE, FAKE, None, FAKE, 16, FAKE, None)
     assert st == _lib.GPTQ_EWORKSPACE
     assert lib.gptq_selftest_wait_timeout(FAKE, 0, None) == _lib.GPTQ_EINVAL
+
+
+def test_w4a16_entry_points_reject_bad_arguments(built_lib):
+    lib = _lib.load()
+    BF, F32 = _lib.GPTQ_BF16, _lib.GPTQ_FP32
+    pack = lib.gptq_pack_codes_4bit
+    assert pack(None, 4, 64, 64, FAKE, None, None) == _lib.GPTQ_EINVAL
+    assert pack(None, 0, 64, 64, None, None, None) == _lib.GPTQ_OK          # empty, no buffers
+    assert pack(FAKE, 4, 60, 64, FAKE, None, None) == _lib.GPTQ_EINVAL      # cols % 8
+    assert pack(FAKE, 4, 64, 60, FAKE, None, None) == _lib.GPTQ_EINVAL      # ldc < cols
+    assert pack(FAKE, 4, 64, 68, FAKE, None, None) == _lib.GPTQ_EINVAL      # ldc % 8
+    assert pack(FAKE, 0, 64, 64, FAKE, None, None) == _lib.GPTQ_OK          # empty: no-op
+    mm = lib.gptq_w4a16_matmul
+
+    def call(rows=64, cols=256, group=128, dtype=BF, n=1, ldx=256, ldy=64, x=FAKE):
+        return mm(FAKE, FAKE, FAKE, rows, cols, group, x, dtype, n, ldx, FAKE, ldy, None, None)
+
+    assert call(x=None) == _lib.GPTQ_EINVAL
+    assert call(cols=240, group=-1, ldx=240) == _lib.GPTQ_EINVAL        # cols % 32
+    assert call(group=64) == _lib.GPTQ_EINVAL                            # group not a 128 multiple
+    assert call(cols=384, group=256, ldx=384) == _lib.GPTQ_EINVAL        # group does not divide
+    assert call(group=0) == _lib.GPTQ_EINVAL
+    assert call(ldx=200) == _lib.GPTQ_EINVAL                             # ldx < cols
+    assert call(ldx=260) == _lib.GPTQ_EINVAL                             # ldx % 8
+    assert call(ldy=10) == _lib.GPTQ_EINVAL                              # ldy < rows
+    assert call(n=-1) == _lib.GPTQ_EINVAL
+    assert call(dtype=F32) == _lib.GPTQ_EUNSUPPORTED
+    assert call(n=17) == _lib.GPTQ_EUNSUPPORTED
+    assert call(cols=(1 << 22) + 128, ldx=(1 << 22) + 128) == _lib.GPTQ_EUNSUPPORTED
+    assert call(rows=0) == _lib.GPTQ_OK and call(n=0) == _lib.GPTQ_OK    # empty: no-op
+    assert call(n=0, x=None) == _lib.GPTQ_OK
+    assert _lib.info_status(_lib.GPTQ_INFO_BAD_CODE) == _lib.GPTQ_EINVAL
