@@ -15,7 +15,9 @@ Extra keys: `roofline` for the dominant kernel (the tensor-core Hessian SYRK, ti
 events on its stream), `e2e` (the same work through the public API from pinned host buffers,
 copies included), `cpu_baseline` (the fp64 oracle on a bounded sample of the same workload,
 extrapolated; rank 0 at N=1 only), `clocks` (nvidia-smi sampled during the timed region) and
-`gpu_launches` (kernels the library enqueued inside the timed region).
+`gpu_launches` (kernels the library enqueued inside the timed region), and `w4a16`: the packed
+4-bit product that consumes the quantizer's codes (decode GEMV, 1 and 8 activation vectors, and the
+packing kernel), timed alone against the HBM roofline (skip it with --no-w4a16).
 `--impl reference` times the fp64 CPU oracle on the same workload instead (bounded samples).
 """
 from __future__ import annotations

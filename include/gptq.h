@@ -258,7 +258,7 @@ gptq_status gptq_pack_codes_4bit(const uint8_t* codes_dev, int64_t rows, int64_t
  * are added in a fixed order, so results are deterministic for a given device and shape.
  * rows == 0 or n == 0 enqueues nothing. Errors: GPTQ_EINVAL (null pointers, cols <= 0,
  * cols % 32 != 0, group rules, ld or alignment rules, n < 0), GPTQ_EUNSUPPORTED (x_dtype other than
- * GPTQ_BF16, n > 16, rows above 2^27, cols above 2^22).
+ * GPTQ_BF16, n > 16, rows above 2^27, cols above 2^22, rows * G of 2^31 or more).
  */
 gptq_status gptq_w4a16_matmul(const uint32_t* packed_dev, const float* scales_dev,
                               const uint8_t* zeros_dev, int64_t rows, int64_t cols, int group,

@@ -172,7 +172,8 @@ gptq_status gptq_w4a16_matmul(const uint32_t* packed_dev, const float* scales_de
   if (ldx < cols || ldx % 8 != 0 || ldy < rows) return GPTQ_EINVAL;
   if (x_dtype != GPTQ_BF16) return x_dtype == GPTQ_FP32 ? GPTQ_EUNSUPPORTED : GPTQ_EINVAL;
   if (n > 16) return GPTQ_EUNSUPPORTED;
-  if (rows > (static_cast<int64_t>(1) << 27) || cols > (static_cast<int64_t>(1) << 22))
+  if (rows > (static_cast<int64_t>(1) << 27) || cols > (static_cast<int64_t>(1) << 22) ||
+      rows * (group > 0 ? cols / group : 1) >= (static_cast<int64_t>(1) << 31))
     return GPTQ_EUNSUPPORTED;
   if (rows == 0 || n == 0) return GPTQ_OK;  // empty: the buffers may be absent
   if (packed_dev == nullptr || scales_dev == nullptr || zeros_dev == nullptr || X_dev == nullptr ||

@@ -55,8 +55,12 @@ constexpr int kMt = 16;                          // rows of one mma tile (the mm
 constexpr int kRows = 32;                        // rows of one CTA: two mma tiles per warp
 constexpr int kChunk = 128;                      // columns a warp takes per step: 4 lanes x 32
 constexpr int kStages = 3;                       // TMA ring depth per warp
-constexpr int kStageBytes = kRows * kChunk / 2;  // 32 rows x 64 bytes of codes
+constexpr int kCodeBytes = kRows * kChunk / 2;   // codes of one stage: 32 rows x 64 bytes
+constexpr int kXRowBytes = kChunk * 2;           // one activation row of one stage (bf16)
 constexpr int kMaxWarps = 16;
+
+// Bytes of one ring stage: the code tile, then `xh` activation rows of the same 128 columns.
+__host__ __device__ constexpr int stage_bytes(int xh) { return kCodeBytes + xh * kXRowBytes; }
 
 // D = A * B + C for one m16n8k16 tile, bf16 inputs, fp32 accumulation.
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -93,9 +97,11 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t negz, uint32_t
 }
 
 // y[n][r] = sum_c x[n][c] * s[r, g(c)] * (q[r][c] - z[r, g(c)]) for 32 rows per CTA. Each of
-// the CTA's W warps takes the 128-column chunks w, w + W, w + 2W, ... and streams their codes
-// through its own ring of kStages TMA buffers (one 32 x 128 tile each); the warps' partial sums
-// are added in warp order at the end, so the result does not depend on timing.
+// the CTA's W warps takes the 128-column chunks w, w + W, w + 2W, ... and streams them through
+// its own ring of kStages TMA buffers; a stage holds the 32 x 128 code tile and the matching
+// 128 columns of the first `xh` activation rows (xh >= n, rows past n and columns past `cols`
+// arrive as zeros). The warps' partial sums are added in warp order at the end, so the result
+// does not depend on timing.
 //
 // Per chunk and warp, lane (g = lane / 4, t = lane % 4) holds 32 codes (columns 32t .. 32t + 31
 // of the chunk) of each of the rows g, g + 8 (mma tile 0) and g + 16, g + 24 (mma tile 1), and
@@ -105,26 +111,26 @@ __device__ __forceinline__ void dequant_word(uint32_t w, uint32_t negz, uint32_t
 // ({2, 6, 3, 7}), which is the order the nibble pairs come out of dequant_word.
 // Eight steps cover the chunk; its sum is then scaled by the row's group scale in fp32.
 // The group of chunk ch is (ch * gmul) >> 32 with gmul = ceil(2^32 / (group / 128)) -- exact for
-// the sizes the host admits -- and gmul = 0 for one scale per row.
-// Activation rows n >= n_act read row n_act - 1 (their products land in output columns that are
-// never stored); columns past `cols` (a ragged last chunk) read zeros.
+// the sizes the host admits -- and gmul = 0 for one scale per row. Zero points are fetched one
+// chunk ahead. Lanes whose vector n is past xh read row xh - 1 (their products land
+// in output columns that are never stored).
 template <int NT>
-__global__ void __launch_bounds__(kMaxWarps * 32) __maxnreg__(NT == 1 ? 72 : 128)
-w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const float* __restrict__ scales,
-                  const uint8_t* __restrict__ zeros, int rows, int cols, uint64_t gmul,
-                  int n_groups, const __nv_bfloat16* __restrict__ x, int n_act, int64_t ldx,
+__global__ void __launch_bounds__(kMaxWarps * 32) __maxnreg__(NT == 1 ? 80 : 128)
+w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const __grid_constant__ CUtensorMap tx,
+                  int xh, const float* __restrict__ scales, const uint8_t* __restrict__ zeros,
+                  int rows, int cols, uint64_t gmul, int n_groups, int n_act,
                   float* __restrict__ y, int64_t ldy, int32_t* info) {
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ volatile int abort_flag;
   const int nwarps = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  uint8_t* ring = smem + warp * (kStages * kStageBytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + nwarps * (kStages * kStageBytes)) +
+  const int sbytes = stage_bytes(xh);
+  uint8_t* ring = smem + warp * (kStages * sbytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + nwarps * (kStages * sbytes)) +
                    warp * kStages;
   const int row0 = blockIdx.x * kRows;
   const int nchunks = (cols + kChunk - 1) / kChunk;
-  const int full_chunks = cols / kChunk;
 
   if (lane == 0) {
 #pragma unroll
@@ -138,28 +144,26 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const float* __res
   int issued = 0;  // loads this warp has started (lane 0's count)
   if (lane == 0) {
     prefetch_tmap(&tcodes);
+    prefetch_tmap(&tx);
     for (int s = 0; s < kStages; ++s) {
       const int ch = warp + s * nwarps;
       if (ch >= nchunks) break;
-      mbar_arrive_expect_tx(&bars[s], kStageBytes);
-      tma_load_2d(ring + s * kStageBytes, &tcodes, &bars[s], ch * (kChunk / 8), row0);
+      mbar_arrive_expect_tx(&bars[s], sbytes);
+      tma_load_2d(ring + s * sbytes, &tcodes, &bars[s], ch * (kChunk / 8), row0);
+      tma_load_2d(ring + s * sbytes + kCodeBytes, &tx, &bars[s], ch * kChunk, 0);
       ++issued;
     }
   }
 
-  // Rows past the end read the last row's metadata (their results are not stored).
-  const float* srow[4];
-  const uint8_t* zrow[4];
+  // Offsets of this lane's four rows in the [rows x n_groups] metadata (below 2^31: the host
+  // checks); rows past the end read the last row's (their results are not stored).
+  int moff[4];
 #pragma unroll
-  for (int m = 0; m < 4; ++m) {
-    const int r = min(row0 + g + 8 * m, rows - 1);
-    srow[m] = scales + static_cast<int64_t>(r) * n_groups;
-    zrow[m] = zeros + static_cast<int64_t>(r) * n_groups;
-  }
-  const __nv_bfloat16* xl[NT];
+  for (int m = 0; m < 4; ++m) moff[m] = min(row0 + g + 8 * m, rows - 1) * n_groups;
+  int xoff[NT];  // byte offset of this lane's activations inside a stage
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt)
-    xl[nt] = x + static_cast<int64_t>(min(nt * 8 + g, n_act - 1)) * ldx + 32 * t;
+    xoff[nt] = kCodeBytes + min(nt * 8 + g, xh - 1) * kXRowBytes + 64 * t;
 
   float acc[2][NT][4];
 #pragma unroll
@@ -169,6 +173,14 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const float* __res
 #pragma unroll
       for (int e = 0; e < 4; ++e) acc[h][nt][e] = 0.f;
 
+  // zero points of the chunk about to be consumed
+  uint32_t zq[4];
+  {
+    const uint32_t gi = static_cast<uint32_t>((static_cast<uint64_t>(warp) * gmul) >> 32);
+#pragma unroll
+    for (int m = 0; m < 4; ++m) zq[m] = __ldg(zeros + moff[m] + gi);
+  }
+
   bool ok = true;
   int j = 0;  // chunks this warp has consumed
   uint32_t phase = 0;
@@ -177,27 +189,21 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const float* __res
     for (int s = 0; s < kStages; ++s) {
       const int ch = base + s * nwarps;
       if (ch >= nchunks) break;
+      // scales of this chunk (first needed after its products), zero points of the next chunk
+      // of this warp (clamped: the last chunk reloads its own)
       const uint32_t gi = static_cast<uint32_t>((static_cast<uint64_t>(ch) * gmul) >> 32);
+      const int chn = min(ch + nwarps, nchunks - 1);
+      const uint32_t gin = static_cast<uint32_t>((static_cast<uint64_t>(chn) * gmul) >> 32);
       float sc[4];
-      uint32_t nz[4];
+      uint32_t zq_n[4];
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
-        sc[m] = __ldg(srow[m] + gi);
-        nz[m] = (0xC300u + __ldg(zrow[m] + gi)) * 0x00010001u;  // -(128 + z), twice
+        sc[m] = __ldg(scales + moff[m] + gi);
+        zq_n[m] = __ldg(zeros + moff[m] + gin);
       }
-      uint4 xv[NT][4];
+      uint32_t nz[4];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const uint4* xp = reinterpret_cast<const uint4*>(xl[nt] + ch * kChunk);
-        if (ch < full_chunks) {
-#pragma unroll
-          for (int i = 0; i < 4; ++i) xv[nt][i] = __ldg(xp + i);
-        } else {
-          const bool in_cols = ch * kChunk + 32 * t < cols;
-#pragma unroll
-          for (int i = 0; i < 4; ++i) xv[nt][i] = in_cols ? __ldg(xp + i) : make_uint4(0, 0, 0, 0);
-        }
-      }
+      for (int m = 0; m < 4; ++m) nz[m] = (0xC300u + zq[m]) * 0x00010001u;  // -(128 + z), twice
 
       const bool got = __all_sync(0xffffffffu,
                                   mbar_wait_bounded(&bars[s], phase, &abort_flag, info));
@@ -205,10 +211,11 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const float* __res
         ok = false;
         break;
       }
-      const uint8_t* st = ring + s * kStageBytes + g * 64 + t * 16;
+      const uint8_t* st = ring + s * sbytes;
       uint4 wv[4];
 #pragma unroll
-      for (int m = 0; m < 4; ++m) wv[m] = *reinterpret_cast<const uint4*>(st + m * 8 * 64);
+      for (int m = 0; m < 4; ++m)
+        wv[m] = *reinterpret_cast<const uint4*>(st + (g + 8 * m) * 64 + t * 16);
 
       float d[2][NT][4];
 #pragma unroll
@@ -222,7 +229,8 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const float* __res
         uint32_t b[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
-          const uint4 v = xv[nt][i];  // x[8i .. 8i+7] of this lane's columns, natural order
+          // x[8i .. 8i+7] of this lane's columns, natural order
+          const uint4 v = *reinterpret_cast<const uint4*>(st + xoff[nt] + 16 * i);
           b[nt][0] = __byte_perm(v.x, v.z, 0x5410);  // (x0, x4)
           b[nt][1] = __byte_perm(v.x, v.z, 0x7632);  // (x1, x5)
           b[nt][2] = __byte_perm(v.y, v.w, 0x5410);  // (x2, x6)
@@ -253,16 +261,20 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const float* __res
           acc[h][nt][2] = fmaf(sc[2 * h + 1], d[h][nt][2], acc[h][nt][2]);
           acc[h][nt][3] = fmaf(sc[2 * h + 1], d[h][nt][3], acc[h][nt][3]);
         }
+#pragma unroll
+      for (int m = 0; m < 4; ++m) zq[m] = zq_n[m];
       ++j;
 
-      // Every lane has consumed stage s (its codes fed the products above): refill it.
+      // Every lane has consumed stage s (its codes and activations fed the products above):
+      // refill it.
       __syncwarp();
       if (lane == 0) {
         const int nxt = ch + kStages * nwarps;
         if (nxt < nchunks) {
           fence_proxy_async_smem();
-          mbar_arrive_expect_tx(&bars[s], kStageBytes);
-          tma_load_2d(ring + s * kStageBytes, &tcodes, &bars[s], nxt * (kChunk / 8), row0);
+          mbar_arrive_expect_tx(&bars[s], sbytes);
+          tma_load_2d(ring + s * sbytes, &tcodes, &bars[s], nxt * (kChunk / 8), row0);
+          tma_load_2d(ring + s * sbytes + kCodeBytes, &tx, &bars[s], nxt * kChunk, 0);
           ++issued;
         }
       }
@@ -297,43 +309,54 @@ w4a16_gemv_kernel(const __grid_constant__ CUtensorMap tcodes, const float* __res
     if (n >= n_act || r >= rows) continue;
     float sum = 0.f;
     for (int w = 0; w < nwarps; ++w)
-      sum += reinterpret_cast<const float*>(smem + w * (kStages * kStageBytes))[row * kLd + n];
+      sum += reinterpret_cast<const float*>(smem + w * (kStages * sbytes))[row * kLd + n];
     y[static_cast<int64_t>(n) * ldy + r] = sum;
   }
 }
 
-size_t gemv_smem_bytes(int nwarps) {
-  return static_cast<size_t>(nwarps) * kStages * (kStageBytes + 8);
+size_t gemv_smem_bytes(int nwarps, int xh) {
+  return static_cast<size_t>(nwarps) * kStages * (stage_bytes(xh) + 8);
 }
 
 // Warps per CTA for a layer of `ctas` CTAs: the most warps per CTA whose CTAs all fit on the
 // device at once (no second, partial wave of CTAs at the end); if no choice fits them all, the one
 // with the most warps resident. Occupancy per warp count comes from the runtime (registers and
-// shared memory of the kernel as built) and is cached per device.
+// shared memory of the kernel as built) and is cached per device and activation tile height.
 template <int NT>
-int pick_warps(int64_t ctas, int64_t nchunks) {
-  static int occ[64][kMaxWarps + 1] = {};
+int pick_warps(int64_t ctas, int64_t nchunks, int xh) {
+  static int occ[64][5][kMaxWarps + 1] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
-  if (occ[dev][0] == 0) {
+  const int xi = xh <= 1 ? 0 : xh <= 2 ? 1 : xh <= 4 ? 2 : xh <= 8 ? 3 : 4;
+  if (occ[dev][xi][0] == 0) {
+    // dynamic shared memory allowed per CTA: the opt-in limit less the kernel's static part
+    int optin = 0;
+    cudaFuncAttributes fa;
+    if (cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+            cudaSuccess ||
+        cudaFuncGetAttributes(&fa, w4a16_gemv_kernel<NT>) != cudaSuccess)
+      return -1;
+    const size_t limit = static_cast<size_t>(optin) - fa.sharedSizeBytes;
     if (cudaFuncSetAttribute(w4a16_gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(gemv_smem_bytes(kMaxWarps))) != cudaSuccess)
+                             static_cast<int>(limit)) != cudaSuccess)
       return -1;
     for (int w = 1; w <= kMaxWarps; ++w) {
       int b = 0;
-      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, w4a16_gemv_kernel<NT>, 32 * w,
-                                                        gemv_smem_bytes(w)) != cudaSuccess)
+      const size_t sm = gemv_smem_bytes(w, xh);
+      if (sm > limit) break;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, w4a16_gemv_kernel<NT>, 32 * w, sm) !=
+          cudaSuccess)
         return -1;
-      occ[dev][w] = b;
+      occ[dev][xi][w] = b;
     }
-    occ[dev][0] = 1;
+    occ[dev][xi][0] = 1;
   }
   const int64_t sms = num_sms();
-  int best = 1;
+  int best = 0;
   int64_t best_resident = -1;
   bool best_fits = false;
   for (int w = 1; w <= kMaxWarps && w <= nchunks; ++w) {
-    const int64_t slots = static_cast<int64_t>(occ[dev][w]) * sms;
+    const int64_t slots = static_cast<int64_t>(occ[dev][xi][w]) * sms;
     if (slots <= 0) continue;
     const bool fits = ctas <= slots;
     const int64_t resident = (fits ? ctas : slots) * w;
@@ -347,16 +370,17 @@ int pick_warps(int64_t ctas, int64_t nchunks) {
 }
 
 template <int NT>
-gptq_status launch_gemv(const CUtensorMap& tmap, int64_t rows, int64_t cols, const float* scales,
-                        const uint8_t* zeros, uint64_t gmul, int n_groups,
-                        const __nv_bfloat16* x, int n, int64_t ldx, float* y, int64_t ldy,
-                        int32_t* info, cudaStream_t stream) {
+gptq_status launch_gemv(const CUtensorMap& tcodes, const CUtensorMap& tx, int xh, int64_t rows,
+                        int64_t cols, const float* scales, const uint8_t* zeros, uint64_t gmul,
+                        int n_groups, int n, float* y, int64_t ldy, int32_t* info,
+                        cudaStream_t stream) {
   const int64_t ctas = (rows + kRows - 1) / kRows;
-  const int nwarps = pick_warps<NT>(ctas, (cols + kChunk - 1) / kChunk);
+  const int nwarps = pick_warps<NT>(ctas, (cols + kChunk - 1) / kChunk, xh);
   if (nwarps <= 0) return GPTQ_ECUDA;
   return launch_pdl(w4a16_gemv_kernel<NT>, dim3(static_cast<unsigned>(ctas)), dim3(nwarps * 32),
-                    gemv_smem_bytes(nwarps), stream, tmap, scales, zeros, static_cast<int>(rows),
-                    static_cast<int>(cols), gmul, n_groups, x, n, ldx, y, ldy, info);
+                    gemv_smem_bytes(nwarps, xh), stream, tcodes, tx, xh, scales, zeros,
+                    static_cast<int>(rows), static_cast<int>(cols), gmul, n_groups, n, y, ldy,
+                    info);
 }
 
 }  // namespace
@@ -375,9 +399,14 @@ gptq_status run_w4a16_gemv(const uint32_t* packed, const float* scales, const ui
                            int64_t rows, int64_t cols, int group, const void* x, int64_t n,
                            int64_t ldx, float* y, int64_t ldy, int32_t* info,
                            cudaStream_t stream) {
-  CUtensorMap tmap;
-  gptq_status st = encode_tmap_2d(&tmap, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, 4, cols / 8,
+  // Activation tile height: n rounded up to a power of two (rows past n arrive as zeros).
+  const int xh = n <= 1 ? 1 : n <= 2 ? 2 : n <= 4 ? 4 : n <= 8 ? 8 : 16;
+  CUtensorMap tcodes, tx;
+  gptq_status st = encode_tmap_2d(&tcodes, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, 4, cols / 8,
                                   rows, cols / 8, kChunk / 8, kRows, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != GPTQ_OK) return st;
+  st = encode_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, 2, cols, n, ldx, kChunk, xh,
+                      CU_TENSOR_MAP_SWIZZLE_NONE);
   if (st != GPTQ_OK) return st;
   const int n_groups = group > 0 ? static_cast<int>(cols / group) : 1;
   // chunk -> group index as (chunk * gmul) >> 32 with gmul = ceil(2^32 / d), d = group / 128
@@ -385,12 +414,11 @@ gptq_status run_w4a16_gemv(const uint32_t* packed, const float* scales, const ui
   // maps every chunk to group 0 (one scale per row).
   const uint64_t d = group > 0 ? static_cast<uint64_t>(group / kChunk) : 0;
   const uint64_t gmul = d == 0 ? 0 : ((1ull << 32) + d - 1) / d;
-  const auto* xb = static_cast<const __nv_bfloat16*>(x);
   if (n <= 8)
-    return launch_gemv<1>(tmap, rows, cols, scales, zeros, gmul, n_groups, xb,
-                          static_cast<int>(n), ldx, y, ldy, info, stream);
-  return launch_gemv<2>(tmap, rows, cols, scales, zeros, gmul, n_groups, xb, static_cast<int>(n),
-                        ldx, y, ldy, info, stream);
+    return launch_gemv<1>(tcodes, tx, xh, rows, cols, scales, zeros, gmul, n_groups,
+                          static_cast<int>(n), y, ldy, info, stream);
+  return launch_gemv<2>(tcodes, tx, xh, rows, cols, scales, zeros, gmul, n_groups,
+                        static_cast<int>(n), y, ldy, info, stream);
 }
 
 }  // namespace gptq
