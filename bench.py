@@ -17,7 +17,9 @@ copies included), `cpu_baseline` (the fp64 oracle on a bounded sample of the sam
 extrapolated; rank 0 at N=1 only), `clocks` (nvidia-smi sampled during the timed region) and
 `gpu_launches` (kernels the library enqueued inside the timed region), and `w4a16`: the packed
 4-bit product that consumes the quantizer's codes (decode GEMV, 1 and 8 activation vectors, and the
-packing kernel), timed alone against the HBM roofline (skip it with --no-w4a16).
+packing kernel), timed alone against the HBM roofline (skip it with --no-w4a16), and `rotation`:
+the data-free Hadamard rotation of the layer's calibration input and weights that can precede
+GPTQ, likewise (skip it with --no-rotation).
 `--impl reference` times the fp64 CPU oracle on the same workload instead (bounded samples).
 """
 from __future__ import annotations
@@ -58,6 +60,7 @@ def parse():
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-w4a16", action="store_true")
+    p.add_argument("--no-rotation", action="store_true")
     p.add_argument("--cpu-sample-s", type=float, default=20.0)
     return p.parse_args()
 
@@ -333,6 +336,46 @@ def bench_w4a16(dev, stream, peaks, peaks_src, iters=50):
     return out
 
 
+def bench_rotation(dev, stream, peaks, peaks_src, spec, X, iters=10):
+    """The data-free Hadamard rotation applied before GPTQ, timed alone with CUDA events on the
+    launching stream: the layer's whole calibration input (token-major bf16, rotated into a second
+    buffer of the same size, both far larger than L2) and its fp32 weights. Algorithmic bytes per
+    launch: one read and one write of every element."""
+    import numpy as np
+    import torch
+    from post_weight_quantization_12_b200 import _lib, synth
+
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    rng = np.random.default_rng(123)
+    bits = np.packbits(rng.random(spec.cols) < 0.5, bitorder="little").view("<u4")
+    sign_bits = torch.from_numpy(bits.view(np.int32).copy()).to(dev)
+    W = synth.weights_torch(spec, 1, dev).float()
+    cases = [("calibration X %dx%d bf16 -> bf16" % tuple(X.shape), X, torch.empty_like(X)),
+             ("weights W %dx%d fp32 -> fp32" % tuple(W.shape), W, torch.empty_like(W))]
+    out = {"kernel": "hadamard_rotate_kernel", "bound": "hbm", "peak_gbs": hbm,
+           "block": _lib.hadamard_block(spec.cols),
+           "peak_source": f"{peaks_src} HBM copy (kernel timed alone)", "cases": []}
+    for name, src, dst in cases:
+        for _ in range(3):
+            _lib.hadamard_rotate(src, dst, sign_bits, stream)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(iters):
+            _lib.hadamard_rotate(src, dst, sign_bits, stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        us = a.elapsed_time(b) / iters * 1e3
+        nbytes = float(src.numel() * src.element_size() + dst.numel() * dst.element_size())
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out["cases"].append({"case": name, "us": us, "bytes": nbytes, "achieved_gbs": gbs,
+                             "frac": gbs / hbm})
+    del cases, W
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -495,6 +538,8 @@ def run_ours(args):
 
     if not args.no_w4a16:
         line["w4a16"] = bench_w4a16(dev, stream, peaks, peaks_src)
+    if not args.no_rotation:
+        line["rotation"] = bench_rotation(dev, stream, peaks, peaks_src, spec, X)
 
     # end to end through the public API from pinned host buffers
     if not args.no_e2e:

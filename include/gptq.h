@@ -265,6 +265,37 @@ gptq_status gptq_w4a16_matmul(const uint32_t* packed_dev, const float* scales_de
                               const void* X_dev, gptq_dtype x_dtype, int64_t n, int64_t ldx,
                               float* Y_dev, int64_t ldy, int32_t* info_dev, void* stream);
 
+/*
+ * Data-free randomized Hadamard rotation of the input-channel axis, applied before GPTQ:
+ *   Y = X Q,  Q = diag(s) (I_{n/b} (x) H_b) / sqrt(b),
+ * H_b the Sylvester Hadamard matrix of order b (entry (i, j) = (-1)^popcount(i & j)), b = the
+ * largest power of two dividing n, at most 4096 (gptq_hadamard_block), s_j = -1 where bit j % 32
+ * of sign_bits[j / 32] is set, else +1.
+ *
+ * Source: "OptRot: Mitigating Weight Outliers via Data-Free Rotations for Post-Training
+ * Quantization", Abstract and Figure 1 (rotations fused into the weights and, transposed, into the
+ * activations leave the layer output unchanged and spread weight outliers) and Theorem 3.1 (the
+ * round-to-nearest error bound grows with the weight incoherence). The page learns its rotations;
+ * this is the data-free randomized Hadamard member of the family it compares against. Rotating
+ * both W (rows = output channels) and the token-major calibration X with the same Q gives
+ * W' X'^T = W X^T and H' = Q^T H Q, so GPTQ can then run on (W', X') unchanged.
+ *
+ *   X_dev      [rows x ldx], x_dtype GPTQ_BF16 or GPTQ_FP32; columns 0..n-1 rotated.
+ *   n          multiple of 32.
+ *   sign_bits_dev  n / 32 uint32 words (drawn by the caller), or NULL for s = +1.
+ *   Y_dev      [rows x ldy], y_dtype GPTQ_BF16 (round to nearest even) or GPTQ_FP32. Y may be X
+ *              itself (same dtype and ld); otherwise the two must not overlap.
+ * Arithmetic: fp32 butterflies (log2 b stages), then the 1/sqrt(b) scale (exact for even log2 b);
+ * deterministic. Requirements: X_dev, Y_dev 16-byte aligned; ldx and ldy times the element size
+ * multiples of 16 bytes. rows == 0 enqueues nothing. Errors: GPTQ_EINVAL (shapes, dtypes,
+ * alignment, null pointers, X == Y with different dtype or ld), GPTQ_EUNSUPPORTED (more than
+ * 2^31 - 1 tiles of 4096 elements).
+ */
+int gptq_hadamard_block(int64_t n);
+gptq_status gptq_hadamard_rotate(const void* X_dev, gptq_dtype x_dtype, int64_t rows, int64_t n,
+                                 int64_t ldx, const uint32_t* sign_bits_dev, void* Y_dev,
+                                 gptq_dtype y_dtype, int64_t ldy, void* stream);
+
 /* Workspace bytes needed by one call (GPTQ_WS_PREPARE or GPTQ_WS_QUANTIZE); 0 for bad input. */
 size_t gptq_workspace_size(int which, int64_t rows, int64_t cols, int block);
 

@@ -46,16 +46,29 @@ def rotation_matrix(n: int, signs=None) -> np.ndarray:
 
 
 def rotate(X: np.ndarray, signs=None) -> np.ndarray:
-    """X Q for the rows of X [rows, n] (weights or token-major activations), in fp64."""
+    """X Q for the rows of X [rows, n] (weights or token-major activations), in fp64. Q is block
+    diagonal, so each block of b columns is multiplied by its own diag(signs) H_b / sqrt(b)."""
     X64 = np.asarray(X, dtype=np.float64)
-    return X64 @ rotation_matrix(X64.shape[1], signs)
+    n = X64.shape[1]
+    b = hadamard_block(n)
+    Hb = scipy.linalg.hadamard(b).astype(np.float64) / np.sqrt(b)
+    s = np.ones(n) if signs is None else np.asarray(signs, dtype=np.float64)
+    out = np.empty_like(X64)
+    for k in range(n // b):
+        blk = slice(k * b, (k + 1) * b)
+        out[:, blk] = (X64[:, blk] * s[blk]) @ Hb
+    return out
 
 
 def rotate_abs_terms(X: np.ndarray) -> np.ndarray:
     """sum over the inputs of |x_i| |Q_ij| for every output: the magnitude scale of any summation
-    order's rounding error (used to state tolerances)."""
+    order's rounding error (used to state tolerances). Every entry of a block of Q has magnitude
+    1 / sqrt(b), so this is the block's sum of |x| over sqrt(b), repeated over the block."""
     X64 = np.abs(np.asarray(X, dtype=np.float64))
-    return X64 @ np.abs(rotation_matrix(X64.shape[1]))
+    n = X64.shape[1]
+    b = hadamard_block(n)
+    sums = X64.reshape(X64.shape[0], n // b, b).sum(axis=2) / np.sqrt(b)
+    return np.repeat(sums, b, axis=1)
 
 
 def weight_incoherence(W: np.ndarray) -> float:

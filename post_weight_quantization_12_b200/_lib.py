@@ -38,6 +38,8 @@ SIGNATURES = {
                                            _P, _P, _P, _P, _P, _P]),
     "gptq_kernel_launches": (ctypes.c_uint64, []),
     "gptq_pack_codes_4bit": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "gptq_hadamard_block": (_I32, [_I64]),
+    "gptq_hadamard_rotate": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I32, _I64, _P]),
     "gptq_w4a16_matmul": (_I32, [_P, _P, _P, _I64, _I64, _I32, _P, _I32, _I64, _I64, _P, _I64, _P,
                                  _P]),
     "gptq_selftest_gemm": (_I32, [_P, _I64, _I32, _P, _I64, _I32, _P, _I64, _I32, _I32, _I32,
@@ -193,6 +195,23 @@ def w4a16_matmul(packed, scales, zeros, group, X, Y, info=None, stream=None):
                                   8 * packed.shape[1], int(group), _ptr(X), _dtype_code(X),
                                   X.shape[0], ldx, _ptr(Y), ldy, _ptr(info), _stream(stream))
     _check(st, "gptq_w4a16_matmul")
+
+
+def hadamard_block(n: int) -> int:
+    """Order b of the Hadamard blocks the rotation uses for width n (0 for n <= 0)."""
+    return int(load().gptq_hadamard_block(int(n)))
+
+
+def hadamard_rotate(X, Y, sign_bits=None, stream=None):
+    """Y[rows, n] = X[rows, n] Q (bf16 or fp32 each; Y may be X). sign_bits: int32/uint32 tensor
+    of n // 32 words (bit j % 32 of word j // 32 set: column j negated) or None."""
+    ldx, ldy = _row_major_ld(X, "X"), _row_major_ld(Y, "Y")
+    if X.shape != Y.shape:
+        raise ValueError("X and Y must have the same shape")
+    st = load().gptq_hadamard_rotate(_ptr(X), _dtype_code(X), X.shape[0], X.shape[1], ldx,
+                                     _ptr(sign_bits), _ptr(Y), _dtype_code(Y), ldy,
+                                     _stream(stream))
+    _check(st, "gptq_hadamard_rotate")
 
 
 def selftest_gemm(A, a_mn, B, b_mn, C, M, N, K, alpha=1.0, beta=0.0, lower=False,

@@ -184,6 +184,25 @@ gptq_status gptq_w4a16_matmul(const uint32_t* packed_dev, const float* scales_de
                         ldy, info_dev, static_cast<cudaStream_t>(stream));
 }
 
+int gptq_hadamard_block(int64_t n) { return hadamard_block_order(n); }
+
+gptq_status gptq_hadamard_rotate(const void* X_dev, gptq_dtype x_dtype, int64_t rows, int64_t n,
+                                 int64_t ldx, const uint32_t* sign_bits_dev, void* Y_dev,
+                                 gptq_dtype y_dtype, int64_t ldy, void* stream) {
+  if (rows < 0 || n <= 0 || n % 32 != 0 || ldx < n || ldy < n) return GPTQ_EINVAL;
+  if ((x_dtype != GPTQ_BF16 && x_dtype != GPTQ_FP32) ||
+      (y_dtype != GPTQ_BF16 && y_dtype != GPTQ_FP32))
+    return GPTQ_EINVAL;
+  const int64_t xe = x_dtype == GPTQ_BF16 ? 2 : 4, ye = y_dtype == GPTQ_BF16 ? 2 : 4;
+  if ((ldx * xe) % 16 != 0 || (ldy * ye) % 16 != 0) return GPTQ_EINVAL;
+  if (rows == 0) return GPTQ_OK;  // empty: the buffers may be absent
+  if (X_dev == nullptr || Y_dev == nullptr) return GPTQ_EINVAL;
+  if (!aligned(X_dev, 16) || !aligned(Y_dev, 16) || !aligned(sign_bits_dev, 4)) return GPTQ_EINVAL;
+  if (X_dev == Y_dev && (x_dtype != y_dtype || ldx != ldy)) return GPTQ_EINVAL;
+  return run_hadamard_rotate(X_dev, x_dtype == GPTQ_BF16, ldx, rows, n, sign_bits_dev, Y_dev,
+                             y_dtype == GPTQ_BF16, ldy, static_cast<cudaStream_t>(stream));
+}
+
 size_t gptq_workspace_size(int which, int64_t rows, int64_t cols, int block) {
   if (cols <= 0) return 0;
   if (which == GPTQ_WS_PREPARE) return prepare_workspace_bytes(cols);

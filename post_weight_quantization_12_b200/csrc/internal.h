@@ -83,6 +83,12 @@ gptq_status run_w4a16_gemv(const uint32_t* packed, const float* scales, const ui
                            int64_t rows, int64_t cols, int group, const void* x, int64_t n,
                            int64_t ldx, float* y, int64_t ldy, int32_t* info, cudaStream_t stream);
 
+// Randomized Hadamard rotation of the rows' input-channel axis (rotation.cu).
+int hadamard_block_order(int64_t n);
+gptq_status run_hadamard_rotate(const void* X, int x_bf16, int64_t ldx, int64_t rows, int64_t n,
+                                const uint32_t* sign_bits, void* Y, int y_bf16, int64_t ldy,
+                                cudaStream_t stream);
+
 // Host-side count of kernels this library has enqueued (diagnostic, see gptq_kernel_launches).
 void count_launch(uint64_t n = 1);
 

@@ -120,3 +120,23 @@ def test_w4a16_entry_points_reject_bad_arguments(built_lib):
     assert call(rows=0) == _lib.GPTQ_OK and call(n=0) == _lib.GPTQ_OK    # empty: no-op
     assert call(n=0, x=None) == _lib.GPTQ_OK
     assert _lib.info_status(_lib.GPTQ_INFO_BAD_CODE) == _lib.GPTQ_EINVAL
+
+
+def test_rotation_entry_points(built_lib):
+    lib = _lib.load()
+    for n, b in ((4096, 4096), (11008, 256), (12288, 4096), (49152, 4096), (96, 32), (0, 0)):
+        assert _lib.hadamard_block(n) == b
+    BF, F32 = _lib.GPTQ_BF16, _lib.GPTQ_FP32
+    rot = lib.gptq_hadamard_rotate
+
+    def call(rows=4, n=256, ldx=256, xd=BF, yd=BF, ldy=256, x=FAKE, y=ctypes.c_void_p(0x20000)):
+        return rot(x, xd, rows, n, ldx, None, y, yd, ldy, None)
+
+    assert call(n=240, ldx=240, ldy=240) == _lib.GPTQ_EINVAL         # n % 32
+    assert call(ldx=200) == _lib.GPTQ_EINVAL                         # ldx < n
+    assert call(ldx=260) == _lib.GPTQ_EINVAL                         # ldx * 2 % 16
+    assert call(xd=F32, ldx=258) == _lib.GPTQ_EINVAL                 # ldx * 4 % 16
+    assert call(yd=7) == _lib.GPTQ_EINVAL
+    assert call(x=None) == _lib.GPTQ_EINVAL
+    assert call(y=FAKE, yd=F32) == _lib.GPTQ_EINVAL                  # in place, dtype differs
+    assert call(rows=0, x=None, y=None) == _lib.GPTQ_OK              # empty: no-op

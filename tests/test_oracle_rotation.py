@@ -37,6 +37,15 @@ def test_orthogonal_with_signs():
     assert np.allclose(Q @ Q.T, np.eye(96), atol=1e-14)
 
 
+def test_blockwise_rotate_equals_the_full_matrix_product():
+    rng = np.random.default_rng(9)
+    X = rng.standard_normal((5, 96))
+    s = _signs(96, 10)
+    Q = rotation.rotation_matrix(96, s)
+    assert np.allclose(rotation.rotate(X, s), X @ Q, rtol=1e-13, atol=1e-14)
+    assert np.allclose(rotation.rotate_abs_terms(X), np.abs(X) @ np.abs(Q), rtol=1e-13)
+
+
 def _butterfly(v):
     """Unnormalised fast Walsh-Hadamard transform, written out: stage h pairs i and i + h."""
     v = list(map(float, v))
