@@ -10,3 +10,4 @@ from .w4a16 import (  # noqa: F401
 from .rotation import (  # noqa: F401
     hadamard_block, rotation_matrix, rotate, rotate_abs_terms, weight_incoherence,
 )
+from .obq import obq_row, obq_quantize  # noqa: F401
