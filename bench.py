@@ -19,7 +19,8 @@ extrapolated; rank 0 at N=1 only), `clocks` (nvidia-smi sampled during the timed
 4-bit product that consumes the quantizer's codes (decode GEMV, 1 and 8 activation vectors, and the
 packing kernel), timed alone against the HBM roofline (skip it with --no-w4a16), and `rotation`:
 the data-free Hadamard rotation of the layer's calibration input and weights that can precede
-GPTQ, likewise (skip it with --no-rotation).
+GPTQ, likewise (skip it with --no-rotation), and `obq`: the OBQ greedy-order reference against
+GPTQ's fixed order on a 4096 x 128 layer, timed, with both proxy losses (skip it with --no-obq).
 `--impl reference` times the fp64 CPU oracle on the same workload instead (bounded samples).
 """
 from __future__ import annotations
@@ -61,6 +62,7 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-w4a16", action="store_true")
     p.add_argument("--no-rotation", action="store_true")
+    p.add_argument("--no-obq", action="store_true")
     p.add_argument("--cpu-sample-s", type=float, default=20.0)
     return p.parse_args()
 
@@ -376,6 +378,84 @@ def bench_rotation(dev, stream, peaks, peaks_src, spec, X, iters=10):
     return out
 
 
+def bench_obq(dev, stream, rows=4096, cols=128, tokens=32768, iters=3):
+    """OBQ's greedy order against GPTQ's fixed order on a 4096 x 128 layer, 4-bit per row: the
+    proxy Hessian and its damped inverse factor R come from this library's S1-S5 calls on
+    token-major bf16 inputs, H^-1 = R^T R in fp64. Times the OBQ kernel (greedy, and the natural
+    order through the same downdates), and reports the proxy loss sum_r (w_hat - w)^T H_d
+    (w_hat - w) of OBQ, of OBQ in natural order and of the library's GPTQ column loop, plus the
+    relative layer error with the undamped H. fp64 work per row ~ 2 cols^3 (the downdates);
+    the peak is derived, not measured: 148 SMs x 64 fp64 lanes x 1965 MHz = 18.6e12 fp64
+    instructions/s (the downdate's multiply and subtract are separate instructions)."""
+    import torch
+    from post_weight_quantization_12_b200 import _lib, synth
+
+    spec = synth.scaled_spec(synth.ATTN, rows, cols, tokens, group=-1)
+    X = synth.inputs_torch(spec, 21, dev)
+    W = synth.weights_torch(spec, 21, dev).float()
+    S = torch.zeros(cols, cols, device=dev)
+    R = torch.empty(cols, cols, device=dev)
+    info = torch.zeros(1, device=dev, dtype=torch.int32)
+    _lib.hessian_accumulate(S, X, info, stream)
+    ws = torch.empty(_lib.workspace_size(_lib.GPTQ_WS_PREPARE, 0, cols, 0), device=dev,
+                     dtype=torch.uint8)
+    _lib.prepare_hinv(S, R, tokens, spec.damp, ws, info, stream)
+    torch.cuda.synchronize(dev)
+    if int(info.item()) != 0:
+        raise RuntimeError(f"device status {int(info.item())} preparing the OBQ layer")
+    H = S.double()                                     # undamped H = 2 X^T X / N (both triangles)
+    Hinv = (R.double().T @ R.double()).contiguous()
+    Hd = torch.linalg.inv(Hinv)
+
+    outs = {}
+    for name, greedy in (("obq_greedy", True), ("obq_natural", False)):
+        codes = torch.empty(rows, cols, dtype=torch.uint8, device=dev)
+        W_hat = torch.empty(rows, cols, device=dev)
+        _lib.obq_quantize(W, Hinv, 4, codes, W_hat, greedy=greedy, stream=stream)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        a.record(stream)
+        for _ in range(iters):
+            _lib.obq_quantize(W, Hinv, 4, codes, W_hat, greedy=greedy, stream=stream)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        outs[name] = (a.elapsed_time(b) / iters, W_hat)
+    W_g = torch.empty(rows, cols, device=dev)
+    codes = torch.empty(rows, cols, dtype=torch.uint8, device=dev)
+    sc = torch.empty(rows, 1, device=dev)
+    zz = torch.empty(rows, 1, dtype=torch.uint8, device=dev)
+    wsq = torch.empty(_lib.workspace_size(_lib.GPTQ_WS_QUANTIZE, rows, cols, 128), device=dev,
+                      dtype=torch.uint8)
+    _lib.quantize_layer(W, R, 4, -1, 128, W_g, codes, sc, zz, None, wsq, info, stream)
+    torch.cuda.synchronize(dev)
+
+    Wd = W.double()
+
+    def proxy(Wh):
+        dW = Wh.double() - Wd
+        return float(((dW @ Hd) * dW).sum())
+
+    def rel_err(Wh):
+        dW = Wh.double() - Wd
+        return float(((dW @ H) * dW).sum() / ((Wd @ H) * Wd).sum())
+
+    fp64_ops = 2.0 * rows * cols ** 3
+    out = {"layer": f"{rows}x{cols}, 4-bit per row, {tokens} bf16 tokens", "kernel": "obq_rows_kernel",
+           "bound": "alu", "peak": 18.6e12, "peak_unit": "fp64 instructions/s (derived, nominal)"}
+    for name, (ms, Wh) in outs.items():
+        out[name] = {"ms": ms, "weights_per_s": rows * cols / (ms / 1e3),
+                     "fp64_ops_per_s": fp64_ops / (ms / 1e3),
+                     "frac": fp64_ops / (ms / 1e3) / 18.6e12,
+                     "proxy_loss": proxy(Wh), "rel_layer_error": rel_err(Wh)}
+    out["gptq_column_loop"] = {"proxy_loss": proxy(W_g), "rel_layer_error": rel_err(W_g)}
+    out["gptq_over_obq_proxy_loss"] = out["gptq_column_loop"]["proxy_loss"] / \
+        out["obq_greedy"]["proxy_loss"]
+    del X, S
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -540,6 +620,8 @@ def run_ours(args):
         line["w4a16"] = bench_w4a16(dev, stream, peaks, peaks_src)
     if not args.no_rotation:
         line["rotation"] = bench_rotation(dev, stream, peaks, peaks_src, spec, X)
+    if not args.no_obq:
+        line["obq"] = bench_obq(dev, stream)
 
     # end to end through the public API from pinned host buffers
     if not args.no_e2e:

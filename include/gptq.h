@@ -296,6 +296,42 @@ gptq_status gptq_hadamard_rotate(const void* X_dev, gptq_dtype x_dtype, int64_t 
                                  int64_t ldx, const uint32_t* sign_bits_dev, void* Y_dev,
                                  gptq_dtype y_dtype, int64_t ldy, void* stream);
 
+/*
+ * OBQ: greedy-order quantization of small layers with explicit inverse-Hessian downdates, the
+ * reference that GPTQ's fixed left-to-right order is measured against.
+ *
+ * Source: "Part 2: Adaptive Rounding: Optimal Brain Quantizer (OBQ)", sections "Greedy Search"
+ * (each step quantizes the remaining weight whose quantization raises the proxy loss least,
+ * (w_p - q_p)^2 / H^-1[p, p] up to a factor 2), "Generalized Weight Update" (the other weights
+ * move by -(w_p - q_p) H^-1[:, p] / H^-1[p, p]), "The OBS / GPTQ Trick" (H^-1 loses weight p by
+ * the rank-1 downdate H^-1 - H^-1[:, p] H^-1[p, :] / H^-1[p, p]) and "Limitations of OBQ" (each row
+ * needs its own H^-1, which is why this reference is limited to small layers).
+ *
+ *   W_dev       float32 [rows x ldw], columns 0..cols-1; not modified.
+ *   cols        1 .. 128.
+ *   Hinv_dev    float64 [cols x cols], ld = cols: the symmetric inverse of the damped Hessian
+ *               shared by all rows (e.g. R^T R from gptq_prepare_hinv, in fp64).
+ *   bits        2 .. 8; one grid per row from the original W (GPTQ's per-row grid: min/max with 0
+ *               included, float32, round half to even).
+ *   order_mode  GPTQ_OBQ_GREEDY (OBQ) or GPTQ_OBQ_NATURAL (left to right: GPTQ's order with the
+ *               same explicit downdates).
+ * Outputs (rows x cols, ld = cols): codes_dev uint8, W_hat_dev float32 = s (q - z); order_dev
+ * int32 (column quantized at each step; may be NULL); loss_dev float64 [rows] = sum over the steps
+ * of (w_p - q_p)^2 / H^-1[p, p], which equals (w_hat - w)^T H_d (w_hat - w) (may be NULL);
+ * scales_dev float32 [rows] and zeros_dev uint8 [rows] (may be NULL).
+ * Arithmetic: fp64 for the weights and H^-1, each operation rounded once in a fixed order (no fused
+ * multiply-adds); greedy ties go to the lowest column. Results are reproducible operation by
+ * operation. rows == 0 enqueues nothing. Errors: GPTQ_EINVAL (shapes, bits, mode, null pointers),
+ * GPTQ_EUNSUPPORTED (cols > 128).
+ */
+#define GPTQ_OBQ_NATURAL 0
+#define GPTQ_OBQ_GREEDY 1
+gptq_status gptq_obq_quantize(const float* W_dev, int64_t rows, int64_t cols, int64_t ldw,
+                              const double* Hinv_dev, int bits, int order_mode,
+                              uint8_t* codes_dev, float* W_hat_dev, int32_t* order_dev,
+                              double* loss_dev, float* scales_dev, uint8_t* zeros_dev,
+                              void* stream);
+
 /* Workspace bytes needed by one call (GPTQ_WS_PREPARE or GPTQ_WS_QUANTIZE); 0 for bad input. */
 size_t gptq_workspace_size(int which, int64_t rows, int64_t cols, int block);
 

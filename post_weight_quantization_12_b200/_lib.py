@@ -21,6 +21,7 @@ GPTQ_INFO_BAD_CODE = -3
 GPTQ_WS_PREPARE, GPTQ_WS_QUANTIZE = 1, 2
 GPTQ_ROUTE_DEFAULT, GPTQ_ROUTE_THREE_STEP, GPTQ_ROUTE_REVERSED = 0, 1, 2
 GPTQ_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
+GPTQ_OBQ_NATURAL, GPTQ_OBQ_GREEDY = 0, 1
 
 # name -> (restype, argtypes)
 _P, _I64, _I32, _F, _SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -39,6 +40,8 @@ SIGNATURES = {
     "gptq_kernel_launches": (ctypes.c_uint64, []),
     "gptq_pack_codes_4bit": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "gptq_hadamard_block": (_I32, [_I64]),
+    "gptq_obq_quantize": (_I32, [_P, _I64, _I64, _I64, _P, _I32, _I32, _P, _P, _P, _P, _P, _P,
+                                 _P]),
     "gptq_hadamard_rotate": (_I32, [_P, _I32, _I64, _I64, _I64, _P, _P, _I32, _I64, _P]),
     "gptq_w4a16_matmul": (_I32, [_P, _P, _P, _I64, _I64, _I32, _P, _I32, _I64, _I64, _P, _I64, _P,
                                  _P]),
@@ -212,6 +215,19 @@ def hadamard_rotate(X, Y, sign_bits=None, stream=None):
                                      _ptr(sign_bits), _ptr(Y), _dtype_code(Y), ldy,
                                      _stream(stream))
     _check(st, "gptq_hadamard_rotate")
+
+
+def obq_quantize(W, Hinv, bits, codes, W_hat, order=None, loss=None, scales=None, zeros=None,
+                 greedy=True, stream=None):
+    """OBQ on W[rows, cols <= 128] (fp32) with the shared fp64 inverse Hessian Hinv[cols, cols];
+    outputs are caller tensors (codes uint8 / W_hat fp32 [rows, cols], order int32 [rows, cols],
+    loss fp64 [rows], scales fp32 / zeros uint8 [rows]; the last four optional)."""
+    ldw = _row_major_ld(W, "W")
+    st = load().gptq_obq_quantize(
+        _ptr(W), W.shape[0], W.shape[1], ldw, _ptr(Hinv), int(bits),
+        GPTQ_OBQ_GREEDY if greedy else GPTQ_OBQ_NATURAL, _ptr(codes), _ptr(W_hat), _ptr(order),
+        _ptr(loss), _ptr(scales), _ptr(zeros), _stream(stream))
+    _check(st, "gptq_obq_quantize")
 
 
 def selftest_gemm(A, a_mn, B, b_mn, C, M, N, K, alpha=1.0, beta=0.0, lower=False,

@@ -203,6 +203,22 @@ gptq_status gptq_hadamard_rotate(const void* X_dev, gptq_dtype x_dtype, int64_t 
                              y_dtype == GPTQ_BF16, ldy, static_cast<cudaStream_t>(stream));
 }
 
+gptq_status gptq_obq_quantize(const float* W_dev, int64_t rows, int64_t cols, int64_t ldw,
+                              const double* Hinv_dev, int bits, int order_mode,
+                              uint8_t* codes_dev, float* W_hat_dev, int32_t* order_dev,
+                              double* loss_dev, float* scales_dev, uint8_t* zeros_dev,
+                              void* stream) {
+  if (rows < 0 || cols < 1 || ldw < cols || bits < 2 || bits > 8) return GPTQ_EINVAL;
+  if (order_mode != GPTQ_OBQ_NATURAL && order_mode != GPTQ_OBQ_GREEDY) return GPTQ_EINVAL;
+  if (cols > 128) return GPTQ_EUNSUPPORTED;
+  if (rows == 0) return GPTQ_OK;  // empty: the buffers may be absent
+  if (W_dev == nullptr || Hinv_dev == nullptr || codes_dev == nullptr || W_hat_dev == nullptr)
+    return GPTQ_EINVAL;
+  return run_obq_quantize(W_dev, rows, cols, ldw, Hinv_dev, bits, order_mode == GPTQ_OBQ_GREEDY,
+                          codes_dev, W_hat_dev, order_dev, loss_dev, scales_dev, zeros_dev,
+                          static_cast<cudaStream_t>(stream));
+}
+
 size_t gptq_workspace_size(int which, int64_t rows, int64_t cols, int block) {
   if (cols <= 0) return 0;
   if (which == GPTQ_WS_PREPARE) return prepare_workspace_bytes(cols);

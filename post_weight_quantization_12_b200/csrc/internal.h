@@ -89,6 +89,12 @@ gptq_status run_hadamard_rotate(const void* X, int x_bf16, int64_t ldx, int64_t 
                                 const uint32_t* sign_bits, void* Y, int y_bf16, int64_t ldy,
                                 cudaStream_t stream);
 
+// OBQ greedy-order reference for layers of at most 128 columns (obq.cu).
+gptq_status run_obq_quantize(const float* W, int64_t rows, int64_t cols, int64_t ldw,
+                             const double* Hinv, int bits, int greedy, uint8_t* codes,
+                             float* W_hat, int32_t* order, double* loss, float* scales,
+                             uint8_t* zeros, cudaStream_t stream);
+
 // Host-side count of kernels this library has enqueued (diagnostic, see gptq_kernel_launches).
 void count_launch(uint64_t n = 1);
 

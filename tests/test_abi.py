@@ -140,3 +140,20 @@ def test_rotation_entry_points(built_lib):
     assert call(x=None) == _lib.GPTQ_EINVAL
     assert call(y=FAKE, yd=F32) == _lib.GPTQ_EINVAL                  # in place, dtype differs
     assert call(rows=0, x=None, y=None) == _lib.GPTQ_OK              # empty: no-op
+
+
+def test_obq_entry_point_rejects_bad_arguments(built_lib):
+    lib = _lib.load()
+
+    def call(rows=4, cols=64, ldw=64, bits=4, mode=1, w=FAKE):
+        return lib.gptq_obq_quantize(w, rows, cols, ldw, FAKE, bits, mode, FAKE, FAKE, None, None,
+                                     None, None, None)
+
+    assert call(cols=0) == _lib.GPTQ_EINVAL
+    assert call(ldw=32) == _lib.GPTQ_EINVAL
+    assert call(bits=1) == _lib.GPTQ_EINVAL and call(bits=9) == _lib.GPTQ_EINVAL
+    assert call(mode=2) == _lib.GPTQ_EINVAL
+    assert call(w=None) == _lib.GPTQ_EINVAL
+    assert call(cols=129, ldw=129) == _lib.GPTQ_EUNSUPPORTED
+    assert call(rows=0, w=None) == _lib.GPTQ_OK
+
