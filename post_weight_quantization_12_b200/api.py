@@ -8,6 +8,13 @@
 Host tensors are copied to the device (pinned-memory, non-blocking) before the call; outputs stay
 on the device unless `to_host=True`. PyTorch only provides memory and streams here; every step of
 the method runs in the library's kernels.
+
+A 4-bit result can be packed for the W4A16 product, and weights and calibration inputs can be
+rotated before quantization:
+
+    lin = pack_4bit(out)                      # PackedLinear4: packed codes, scales, zeros
+    Y = lin(X)                                # fp32 [n, rows] = X W_hat^T for bf16 X [n <= 16, cols]
+    Wr, Xr = rotate(W, signs), rotate(X, signs)   # data-free randomized Hadamard rotation
 """
 from __future__ import annotations
 
@@ -144,3 +151,48 @@ class LayerQuantizer:
         else:
             info = int(self.info.item())
         return QuantizedLayer(codes, scales, zeros, W_hat, err_sq, info)
+
+
+@dataclass
+class PackedLinear4:
+    """A 4-bit quantized linear layer in the packed layout the W4A16 product reads."""
+    packed: torch.Tensor     # int32 [rows, cols // 8]: eight 4-bit codes per word
+    scales: torch.Tensor     # fp32 [rows, G]
+    zeros: torch.Tensor      # uint8 [rows, G]
+    group: int               # -1 (per row) or the group size
+
+    @property
+    def rows(self) -> int:
+        return self.packed.shape[0]
+
+    @property
+    def cols(self) -> int:
+        return 8 * self.packed.shape[1]
+
+    def __call__(self, X: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+        """fp32 [n, rows] = X W_hat^T for bf16 activations X [n, cols], n <= 16."""
+        if out is None:
+            out = torch.empty(X.shape[0], self.rows, device=X.device, dtype=torch.float32)
+        _lib.w4a16_matmul(self.packed, self.scales, self.zeros, self.group, X, out, stream=stream)
+        return out
+
+
+def pack_4bit(layer: QuantizedLayer, stream=None) -> PackedLinear4:
+    """Packs the codes of a 4-bit QuantizedLayer (device tensors) for the W4A16 product."""
+    rows, cols = layer.codes.shape
+    G = layer.scales.shape[1]
+    packed = torch.empty(rows, cols // 8, device=layer.codes.device, dtype=torch.int32)
+    _lib.pack_codes_4bit(layer.codes, packed, stream=stream)
+    return PackedLinear4(packed, layer.scales, layer.zeros, -1 if G == 1 else cols // G)
+
+
+def rotate(X: torch.Tensor, sign_bits=None, out=None, stream=None) -> torch.Tensor:
+    """X Q with Q = diag(signs) (I (x) H_b) / sqrt(b), the randomized Hadamard rotation of the last
+    axis (see gptq_hadamard_rotate); `sign_bits` int32 [cols // 32] (bit j % 32 of word j // 32 set
+    negates column j) or None. Returns a new tensor of X's dtype unless `out` is given (which may
+    be X itself)."""
+    if out is None:
+        out = torch.empty_like(X)
+    _lib.hadamard_rotate(X, out, sign_bits, stream)
+    return out
+

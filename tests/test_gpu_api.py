@@ -34,3 +34,36 @@ def test_host_chunks_match_device_inputs():
     s = out_h.scales.numpy().repeat(128, axis=1)
     z = out_h.zeros.numpy().repeat(128, axis=1).astype(np.float32)
     np.testing.assert_array_equal(out_h.W_hat.numpy(), s * (out_h.codes.numpy().astype(np.float32) - z))
+
+
+def test_pack_4bit_linear_reproduces_x_w_hat():
+    """A 4-bit group-128 layer from LayerQuantizer, packed and applied to bf16 activations, gives
+    X W_hat^T within the product's rounding bound."""
+    spec = synth.scaled_spec(synth.ATTN, 96, 512, 4096)
+    X = synth.inputs_torch(spec, 3, DEV)
+    W = synth.weights_torch(spec, 3, DEV)
+    q = api.LayerQuantizer(spec.cols, device=DEV)
+    q.add_batch(X)
+    out = q.quantize(W, bits=4, group=128, block=128)
+    lin = api.pack_4bit(out)
+    assert lin.group == 128 and lin.rows == 96 and lin.cols == 512
+    A = X[:3].contiguous()
+    Y = lin(A)
+    torch.cuda.synchronize()
+    ref = A.double() @ out.W_hat.double().T
+    terms = A.double().abs() @ out.W_hat.double().abs().T
+    bound = 8 * 2.0 ** -22 + (4 + 16) * 2.0 ** -24 + 2.0 ** -23
+    assert torch.all((Y.double() - ref).abs() <= bound * terms)
+
+
+def test_rotate_helper_keeps_layer_products():
+    W = torch.randn(8, 256, generator=torch.Generator().manual_seed(5)).to(DEV)
+    X = torch.randn(32, 256, generator=torch.Generator().manual_seed(6)).to(DEV)
+    signs = torch.randint(-2 ** 31, 2 ** 31 - 1, (8,), generator=torch.Generator().manual_seed(7),
+                          dtype=torch.int64).to(torch.int32).to(DEV)
+    Wr, Xr = api.rotate(W, signs), api.rotate(X, signs)
+    torch.cuda.synchronize()
+    ref = W.double() @ X.double().T
+    scale = W.double().norm(dim=1)[:, None] * X.double().norm(dim=1)[None, :]
+    assert torch.all((Wr.double() @ Xr.double().T - ref).abs() <= 1e-5 * scale)
+
