@@ -3,7 +3,9 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 #include "internal.h"
@@ -25,6 +27,21 @@ __global__ void selftest_wait_kernel(int32_t* info, uint64_t limit_ns) {
   __syncthreads();
   if (threadIdx.x == 0) mbar_wait_bounded(&bar, 0, &abort_flag, info, limit_ns);
   __syncthreads();
+}
+
+gptq_status set_max_dynamic_smem(const void* kernel, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ECUDA;
+  static std::mutex mu;
+  static std::map<std::pair<const void*, int>, int> done;  // (kernel, device) -> bytes set
+  std::lock_guard<std::mutex> lock(mu);
+  auto it = done.find({kernel, dev});
+  if (it != done.end() && it->second >= bytes) return GPTQ_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return GPTQ_ECUDA;
+  done[{kernel, dev}] = bytes;
+  return GPTQ_OK;
 }
 
 int num_sms() {

@@ -732,13 +732,9 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
   if ((st = operand_map(&tAs, g.As, g.lda, g.a_mn, g.M + ext, K + ext)) != GPTQ_OK) return st;
   if ((st = operand_map(&tBb, g.Bb, g.ldb, g.b_mn, g.N + ext, K + ext)) != GPTQ_OK) return st;
   if ((st = operand_map(&tBs, g.Bs, g.ldb, g.b_mn, g.N + ext, K + ext)) != GPTQ_OK) return st;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(gemm_tf32x3_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
-      return GPTQ_ECUDA;
-    attr_done = true;
-  }
+  if ((st = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_tf32x3_tc), kSmemBytes)) !=
+      GPTQ_OK)
+    return st;
   TcGemmParams p;
   p.M = g.M; p.N = g.N; p.K = g.K;
   p.a_mn = g.a_mn; p.b_mn = g.b_mn;
@@ -758,13 +754,9 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
   const bool panel = g.K > 0 && g.K <= tgp::kMaxK && !g.klo_from_m && !g.klo_from_n &&
                      !g.khi_from_m && g.batch == 1 && (!g.lower || g.M == g.N);
   if (panel) {
-    static bool attr_p = false;
-    if (!attr_p) {
-      if (cudaFuncSetAttribute(gemm_tf32x3_panel_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               tgp::kSmemBytesStaged) != cudaSuccess)
-        return GPTQ_ECUDA;
-      attr_p = true;
-    }
+    if ((st = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_tf32x3_panel_tc),
+                                   tgp::kSmemBytesStaged)) != GPTQ_OK)
+      return st;
     const int64_t nt = g.lower ? static_cast<int64_t>(tiles_m) * (tiles_m + 1) / 2
                                : static_cast<int64_t>(tiles_m) * p.tiles_n;
     if (nt > 0x7fffffff) return GPTQ_EUNSUPPORTED;

@@ -300,13 +300,9 @@ gptq_status launch_hessian_bf16(float* S, int64_t cols, const void* X, int64_t n
                                   static_cast<uint64_t>(ldx), kBoxCh, kBK,
                                   CU_TENSOR_MAP_SWIZZLE_128B);
   if (st != GPTQ_OK) return st;
-  static bool attr_done = false;  // benign race: setting the same attribute twice is harmless
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(hessian_syrk_bf16_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             kSmemBytes) != cudaSuccess)
-      return GPTQ_ECUDA;
-    attr_done = true;
-  }
+  if ((st = set_max_dynamic_smem(reinterpret_cast<const void*>(hessian_syrk_bf16_tc),
+                                 kSmemBytes)) != GPTQ_OK)
+    return st;
   // lower 256 x 256 super-tiles, one per CTA pair per round
   const int n_s = static_cast<int>((cols + 255) / 256);
   const int n_super = n_s * (n_s + 1) / 2;

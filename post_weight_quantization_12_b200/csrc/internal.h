@@ -95,6 +95,10 @@ gptq_status run_obq_quantize(const float* W, int64_t rows, int64_t cols, int64_t
                              float* W_hat, int32_t* order, double* loss, float* scales,
                              uint8_t* zeros, cudaStream_t stream);
 
+// Raises a kernel's dynamic shared-memory limit to at least `bytes` on the current device. The
+// attribute belongs to the (kernel, device) pair; each pair is set once, under a lock.
+gptq_status set_max_dynamic_smem(const void* kernel, int bytes);
+
 // Host-side count of kernels this library has enqueued (diagnostic, see gptq_kernel_launches).
 void count_launch(uint64_t n = 1);
 

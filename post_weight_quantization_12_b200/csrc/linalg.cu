@@ -559,13 +559,9 @@ potrf_diag_kernel(float* A, int64_t lda, int k0, int nb, float* Db, float* Ds, i
 static gptq_status launch_potrf_diag(float* A, int64_t n, int k0, int nb, float* Db, float* Ds,
                                      int64_t ldd, int32_t* info, int info_base, int rev_n,
                                      bool store_l, cudaStream_t stream) {
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(potrf_diag_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             la::kDiagSmem) != cudaSuccess)
-      return GPTQ_ECUDA;
-    attr_done = true;
-  }
+  const gptq_status st =
+      set_max_dynamic_smem(reinterpret_cast<const void*>(potrf_diag_kernel), la::kDiagSmem);
+  if (st != GPTQ_OK) return st;
   return launch_pdl(potrf_diag_kernel, dim3(1), dim3(la::kDiagThreads), la::kDiagSmem, stream, A, n,
                     k0, nb, Db, Ds, ldd, info, info_base, rev_n, store_l ? 1 : 0);
 }

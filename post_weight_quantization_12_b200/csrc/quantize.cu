@@ -407,13 +407,9 @@ static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, con
   const int rows_per_cta = THREADS / TPR;
   const int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
   constexpr int smem = (B * B + B) * 4;
-  static bool attr_done = false;
-  if (!attr_done) {
-    if (cudaFuncSetAttribute(column_loop_kernel<B, TPR, THREADS>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return GPTQ_ECUDA;
-    attr_done = true;
-  }
+  const gptq_status st = set_max_dynamic_smem(
+      reinterpret_cast<const void*>(column_loop_kernel<B, TPR, THREADS>), smem);
+  if (st != GPTQ_OK) return st;
   return launch_pdl(column_loop_kernel<B, TPR, THREADS>, dim3(static_cast<unsigned>(grid)),
                     dim3(THREADS), smem, stream, Wh, rows, cols, R, b0, nb, bits, group, group_mode,
                     gi_fixed, scales, zeros, G, codes, Eb, Es, err_sq, Rb, Rs, nrest);

@@ -15,6 +15,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -324,10 +326,12 @@ size_t gemv_smem_bytes(int nwarps, int xh) {
 // shared memory of the kernel as built) and is cached per device and activation tile height.
 template <int NT>
 int pick_warps(int64_t ctas, int64_t nchunks, int xh) {
+  static std::mutex mu;
   static int occ[64][5][kMaxWarps + 1] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return -1;
   const int xi = xh <= 1 ? 0 : xh <= 2 ? 1 : xh <= 4 ? 2 : xh <= 8 ? 3 : 4;
+  std::lock_guard<std::mutex> lock(mu);
   if (occ[dev][xi][0] == 0) {
     // dynamic shared memory allowed per CTA: the opt-in limit less the kernel's static part
     int optin = 0;
@@ -337,8 +341,8 @@ int pick_warps(int64_t ctas, int64_t nchunks, int xh) {
         cudaFuncGetAttributes(&fa, w4a16_gemv_kernel<NT>) != cudaSuccess)
       return -1;
     const size_t limit = static_cast<size_t>(optin) - fa.sharedSizeBytes;
-    if (cudaFuncSetAttribute(w4a16_gemv_kernel<NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(limit)) != cudaSuccess)
+    if (set_max_dynamic_smem(reinterpret_cast<const void*>(w4a16_gemv_kernel<NT>),
+                             static_cast<int>(limit)) != GPTQ_OK)
       return -1;
     for (int w = 1; w <= kMaxWarps; ++w) {
       int b = 0;
