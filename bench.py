@@ -21,6 +21,8 @@ packing kernel), timed alone against the HBM roofline (skip it with --no-w4a16),
 the data-free Hadamard rotation of the layer's calibration input and weights that can precede
 GPTQ, likewise (skip it with --no-rotation), and `obq`: the OBQ greedy-order reference against
 GPTQ's fixed order on a 4096 x 128 layer, timed, with both proxy losses (skip it with --no-obq).
+Each of these three also carries a `cpu_baseline`: the oracle on a bounded sample of its workload
+(rank 0 at N=1, like the headline's).
 `--impl reference` times the fp64 CPU oracle on the same workload instead (bounded samples).
 """
 from __future__ import annotations
@@ -183,6 +185,54 @@ def oracle_sample(W_np, X_np, spec, budget_s: float):
             f"S2-S5 in full at {cols}x{cols} ({t_s25:.2f} s); S6-S8 on {r_sub} of {spec.rows} rows "
             f"({t_s68:.2f} s, x{spec.rows / r_sub:g}); extrapolated {full:.1f} s per layer")
     return full, desc, t_s1 + t_s25 + t_s68
+
+
+def oracle_extras(rows_w4: int = 256, tokens_rot: int = 4096, rows_obq: int = 64):
+    """The fp64 oracle on bounded samples of the extra legs' workloads, extrapolated to the full
+    ones (time ~ rows, tokens or rows): the W4A16 product of the 12288 x 49152 g128 layer on
+    `rows_w4` rows, the rotation of 262144 x 4096 calibration tokens on `tokens_rot` tokens, OBQ
+    of the 4096 x 128 layer on `rows_obq` rows. Inputs are seeded CPU draws of the same shapes.
+    Returns {"w4a16": {...}, "rotation": {...}, "obq": {...}}, each with the extrapolated value in
+    the leg's own unit."""
+    import numpy as np
+    import oracle
+    from post_weight_quantization_12_b200 import synth
+
+    out = {}
+    cols = 49152
+    codes, scales, zeros = synth.w4a16_operands_torch(rows_w4, cols, 128, 5, "cpu")
+    x = synth.inputs_torch(synth.scaled_spec(synth.ATTN, 1, cols, 1), 7, "cpu").float().numpy()
+    words = oracle.pack_codes(codes.numpy())
+    t0 = time.perf_counter()
+    oracle.w4a16_matmul(words, scales.numpy(), zeros.numpy(), 128, x)
+    dt = time.perf_counter() - t0
+    full = dt * 12288 / rows_w4
+    out["w4a16"] = {"value": full * 1e6, "unit": "us per product (n = 1)", "kind": "oracle",
+                    "cores": cpu_threads(),
+                    "sample": f"{rows_w4} of 12288 rows ({dt:.3f} s, x{12288 / rows_w4:g})"}
+    xr = synth.inputs_torch(synth.scaled_spec(synth.ATTN, 1, 4096, tokens_rot), 9, "cpu")
+    xr = xr.float().numpy()
+    signs = np.where(np.random.default_rng(3).random(4096) < 0.5, -1.0, 1.0)
+    t0 = time.perf_counter()
+    oracle.rotate(xr, signs)
+    dt = time.perf_counter() - t0
+    full = dt * 262144 / tokens_rot
+    out["rotation"] = {"value": full * 1e6, "unit": "us per 262144 x 4096 rotation",
+                       "kind": "oracle", "cores": cpu_threads(),
+                       "sample": f"{tokens_rot} of 262144 tokens ({dt:.3f} s, "
+                                 f"x{262144 / tokens_rot:g})"}
+    rng = np.random.default_rng(11)
+    Xo = rng.standard_normal((1024, 128))
+    Hd = oracle.damp(oracle.hessian(Xo))[0]
+    Wo = (rng.standard_normal((rows_obq, 128)) * 0.02).astype(np.float32)
+    t0 = time.perf_counter()
+    oracle.obq_quantize(Wo, np.linalg.inv(Hd), 4)
+    dt = time.perf_counter() - t0
+    full = dt * 4096 / rows_obq
+    out["obq"] = {"value": full * 1e3, "unit": "ms per 4096 x 128 layer (greedy)", "kind": "oracle",
+                  "cores": cpu_threads(),
+                  "sample": f"{rows_obq} of 4096 rows ({dt:.3f} s, x{4096 / rows_obq:g})"}
+    return out
 
 
 def cpu_threads():
@@ -665,6 +715,11 @@ def run_ours(args):
         line["cpu_baseline"] = {"value": rows * cols / full, "unit": UNIT,
                                 "cores": cpu_threads(), "kind": "oracle", "sample": desc,
                                 "sample_wall_s": spent}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        for key, val in oracle_extras().items():
+            if key in line:
+                line[key]["cpu_baseline"] = val
 
     if rank == 0:
         print(json.dumps(line), flush=True)
