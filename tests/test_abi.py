@@ -157,3 +157,24 @@ def test_obq_entry_point_rejects_bad_arguments(built_lib):
     assert call(cols=129, ldw=129) == _lib.GPTQ_EUNSUPPORTED
     assert call(rows=0, w=None) == _lib.GPTQ_OK
 
+
+
+def test_header_compiles_as_c_and_links(built_lib, tmp_path):
+    """include/gptq.h is plain C (C99, pedantic) and a C program links against the library."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_gptq.c"
+    src.write_text('#include "gptq.h"\n#include <stdio.h>\n'
+                   'int main(void) { printf("%s %d\\n", gptq_version(), '
+                   'gptq_hadamard_block(11008)); return 0; }\n')
+    exe = tmp_path / "use_gptq"
+    inc = os.path.join(os.path.dirname(HEADER))
+    libdir = os.path.dirname(built_lib)
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", inc,
+                    str(src), "-o", str(exe), "-L", libdir, "-l:libgptq_b200.so",
+                    "-Wl,-rpath," + libdir], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out[0].count(".") == 2 and out[1] == "256"
