@@ -198,11 +198,15 @@ gptq_status gptq_quantize_layer(const void* W_dev, gptq_dtype w_dtype, int64_t r
  *     returns GPTQ_EWORKSPACE without enqueueing anything; at block 128 a layer of up to
  *     8192 x 8192 fits;
  *   - the first call on each device looks up the array's device address (cudaGetSymbolAddress
- *     with that device current); make that first call before any stream capture;
+ *     with that device current) and keeps it for the life of the process; make that first call
+ *     before any stream capture. After a cudaDeviceReset of that device the kept address is
+ *     stale: do not use this entry point on a device that has been reset;
  *   - all calls in the process share the one array per device and it keeps the last call's
  *     contents (nothing in it needs to start at zero); calls whose work overlaps on the GPU, e.g.
  *     on two streams at once, race on it -- serialize them.
- * Errors: as gptq_quantize_layer, plus GPTQ_EWORKSPACE when the size limit is exceeded.
+ * Errors: the argument checks of gptq_quantize_layer run first and give its codes (GPTQ_EINVAL,
+ * GPTQ_EUNSUPPORTED); a call that passes them but needs more than the built-in scratch returns
+ * GPTQ_EWORKSPACE.
  */
 #define GPTQ_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
 gptq_status gptq_quantize_layer_noalloc(const void* W_dev, gptq_dtype w_dtype, int64_t rows,

@@ -98,6 +98,28 @@ using namespace gptq;
 
 static bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+gptq_status gptq::check_quantize_args(const void* W, gptq_dtype w_dtype, int64_t rows,
+                                      int64_t cols, int64_t ldw, const float* R, int bits,
+                                      int group, int block, const float* W_hat,
+                                      const uint8_t* codes, const float* scales,
+                                      const uint8_t* zeros) {
+  if (W == nullptr || R == nullptr || W_hat == nullptr || codes == nullptr || scales == nullptr ||
+      zeros == nullptr)
+    return GPTQ_EINVAL;
+  if (rows <= 0 || cols <= 0 || ldw < cols) return GPTQ_EINVAL;
+  if (cols % 4 != 0 || !aligned(R, 16) || !aligned(W_hat, 16)) return GPTQ_EINVAL;
+  if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_FP32) return GPTQ_EINVAL;
+  if (bits < 2 || bits > 8) return GPTQ_EINVAL;
+  if (block != 32 && block != 64 && block != 128) return GPTQ_EINVAL;
+  if (group == 0 || group < -1) return GPTQ_EINVAL;
+  if (group > 0 && (cols % group != 0 || !(group % block == 0 || block % group == 0)))
+    return GPTQ_EINVAL;
+  if (cols > 65536 || rows > (static_cast<int64_t>(1) << 30) ||
+      rows * cols > (static_cast<int64_t>(1) << 40))
+    return GPTQ_EUNSUPPORTED;
+  return GPTQ_OK;
+}
+
 extern "C" {
 
 gptq_status gptq_hessian_accumulate(float* S_dev, int64_t cols, const void* X_dev,
@@ -148,20 +170,9 @@ gptq_status gptq_quantize_layer(const void* W_dev, gptq_dtype w_dtype, int64_t r
                                 float* W_hat_dev, uint8_t* codes_dev, float* scales_dev,
                                 uint8_t* zeros_dev, float* err_sq_dev, void* ws_dev,
                                 size_t ws_bytes, int32_t* info_dev, void* stream) {
-  if (W_dev == nullptr || R_dev == nullptr || W_hat_dev == nullptr || codes_dev == nullptr ||
-      scales_dev == nullptr || zeros_dev == nullptr)
-    return GPTQ_EINVAL;
-  if (rows <= 0 || cols <= 0 || ldw < cols) return GPTQ_EINVAL;
-  if (cols % 4 != 0 || !aligned(R_dev, 16) || !aligned(W_hat_dev, 16)) return GPTQ_EINVAL;
-  if (w_dtype != GPTQ_BF16 && w_dtype != GPTQ_FP32) return GPTQ_EINVAL;
-  if (bits < 2 || bits > 8) return GPTQ_EINVAL;
-  if (block != 32 && block != 64 && block != 128) return GPTQ_EINVAL;
-  if (group == 0 || group < -1) return GPTQ_EINVAL;
-  if (group > 0 && (cols % group != 0 || !(group % block == 0 || block % group == 0)))
-    return GPTQ_EINVAL;
-  if (cols > 65536 || rows > (static_cast<int64_t>(1) << 30) ||
-      rows * cols > (static_cast<int64_t>(1) << 40))
-    return GPTQ_EUNSUPPORTED;
+  const gptq_status st = check_quantize_args(W_dev, w_dtype, rows, cols, ldw, R_dev, bits, group,
+                                             block, W_hat_dev, codes_dev, scales_dev, zeros_dev);
+  if (st != GPTQ_OK) return st;
   if (ws_dev == nullptr || ws_bytes < quantize_workspace_bytes(rows, cols, block) ||
       !aligned(ws_dev, 256))
     return GPTQ_EWORKSPACE;

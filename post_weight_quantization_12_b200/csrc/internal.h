@@ -71,6 +71,11 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t cols, int64_t n_total
 
 // S6-S8
 size_t quantize_workspace_bytes(int64_t rows, int64_t cols, int block);
+// Every argument check of gptq_quantize_layer except the workspace's (GPTQ_OK when they pass).
+gptq_status check_quantize_args(const void* W, gptq_dtype w_dtype, int64_t rows, int64_t cols,
+                                int64_t ldw, const float* R, int bits, int group, int block,
+                                const float* W_hat, const uint8_t* codes, const float* scales,
+                                const uint8_t* zeros);
 gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, int64_t cols,
                                int64_t ldw, const float* R, int bits, int group, int block,
                                float* W_hat, uint8_t* codes, float* scales, uint8_t* zeros,

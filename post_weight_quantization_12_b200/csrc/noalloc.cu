@@ -9,7 +9,10 @@
 // The array is a file-scope __device__ variable, so every GPU that loads the library holds
 // GPTQ_NOALLOC_SCRATCH_BYTES of it until the process exits. Host code may not use the array's
 // name as a device pointer (on the host it is only a stand-in symbol); its device address is
-// looked up once per device with cudaGetSymbolAddress, with that device current.
+// looked up once per device with cudaGetSymbolAddress, with that device current, and cached for
+// the life of the process. A cudaDeviceReset destroys the context that holds the array, so the
+// cached address is stale afterwards: this entry point must not be used on a device after it has
+// been reset.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -48,8 +51,12 @@ extern "C" gptq_status gptq_quantize_layer_noalloc(
     const float* R_dev, int bits, int group, int block, float* W_hat_dev, uint8_t* codes_dev,
     float* scales_dev, uint8_t* zeros_dev, float* err_sq_dev, int32_t* info_dev, void* stream) {
   using namespace gptq;
-  if (block != 32 && block != 64 && block != 128) return GPTQ_EINVAL;
-  if (rows <= 0 || cols <= 0) return GPTQ_EINVAL;
+  // The ordinary argument checks come first, so a call that gptq_quantize_layer would refuse for
+  // its arguments is refused here for the same reason; only a valid call that is too large for
+  // the built-in scratch gets GPTQ_EWORKSPACE.
+  const gptq_status bad = check_quantize_args(W_dev, w_dtype, rows, cols, ldw, R_dev, bits, group,
+                                              block, W_hat_dev, codes_dev, scales_dev, zeros_dev);
+  if (bad != GPTQ_OK) return bad;
   const size_t need = quantize_workspace_bytes(rows, cols, block);
   if (need > GPTQ_NOALLOC_SCRATCH_BYTES) return GPTQ_EWORKSPACE;
   void* scratch = nullptr;

@@ -70,13 +70,24 @@ def test_noalloc_matches_workspace_entry_point(call):
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
+    """A valid call that is too large for the built-in scratch is refused before anything is
+    enqueued. Real (small) buffers are passed: the call is refused on its sizes alone, and if the
+    checks were ever reordered the buffers are still valid device memory."""
     lib = _lib.load()
-    fake = ctypes.c_void_p(0x10000)      # never touched: the size check comes first
     cols = 4096
     rows = 1
     while _lib.workspace_size(_lib.GPTQ_WS_QUANTIZE, rows, cols, 128) <= \
             _lib.GPTQ_NOALLOC_SCRATCH_BYTES:
         rows *= 2
-    st = lib.gptq_quantize_layer_noalloc(fake, _lib.GPTQ_BF16, rows, cols, cols, fake, 4, -1, 128,
-                                         fake, fake, fake, fake, None, fake, None)
+    buf = torch.zeros(4096, dtype=torch.float32, device=DEV)
+    p = ctypes.c_void_p(buf.data_ptr())
+    st = lib.gptq_quantize_layer_noalloc(p, _lib.GPTQ_BF16, rows, cols, cols, p, 4, -1, 128,
+                                         p, p, p, p, None, p, None)
     assert st == _lib.GPTQ_EWORKSPACE
+    # A call with invalid arguments is refused for them, as gptq_quantize_layer refuses it.
+    st = lib.gptq_quantize_layer_noalloc(None, _lib.GPTQ_BF16, rows, cols, cols, p, 4, -1, 128,
+                                         p, p, p, p, None, p, None)
+    assert st == _lib.GPTQ_EINVAL
+    st = lib.gptq_quantize_layer_noalloc(p, _lib.GPTQ_BF16, 64, cols, cols, p, 9, -1, 128,
+                                         p, p, p, p, None, p, None)
+    assert st == _lib.GPTQ_EINVAL
