@@ -160,7 +160,8 @@ def check_shapes(cols: int, group: int, block: int):
             raise ValueError("group and block must nest (one a multiple of the other)")
 
 
-def gptq_quantize(W: np.ndarray, R: np.ndarray, bits: int, group: int = -1, block: int = 128) -> dict:
+def gptq_quantize(W: np.ndarray, R: np.ndarray, bits: int, group: int = -1, block: int = 128,
+                  row_grid=None) -> dict:
     """GPTQ column loop in fixed left-to-right order with lazy block updates.
 
     [GPTQ] "Algorithm GPTQ" and "Observation 2: Lazy Batch Updates"; [BLOG-VI] "2. Lazy batch
@@ -169,7 +170,9 @@ def gptq_quantize(W: np.ndarray, R: np.ndarray, bits: int, group: int = -1, bloc
       * q_j = quantize(w_j); e_j = (w_j - q_hat_j) / R_jj; E[:, j-b0] = e_j;
       * the block's later columns: W[:, j+1:b1] -= e_j R[j, j+1:b1]   (kept "in SRAM");
     then the flush W[:, b1:] -= E R[b0:b1, b1:] (one matrix product).
-    Per-row parameters (group <= 0) are taken once from the original W.
+    Per-row parameters (group <= 0) are taken once from the original W. ``row_grid`` = (s, z)
+    supplies them instead (per-row mode only): when W holds only the leading columns of wider
+    rows, the grid of each whole original row is computed by the caller with quant_params.
     Returns codes [r,c] uint8, scales/zeros [r,G] (float32 / uint8), W_hat [r,c] float32,
     err [r,c] fp64 (the e_j), err_sq [r] fp64 = sum_j e_j^2, w_in [r,c] fp64 (the compensated
     value each weight had when it was quantized).
@@ -186,8 +189,10 @@ def gptq_quantize(W: np.ndarray, R: np.ndarray, bits: int, group: int = -1, bloc
     scales = np.zeros((rows, G), F32)
     zeros = np.zeros((rows, G), F32)
     if group <= 0:
-        s, z = quant_params(W, bits)
+        s, z = quant_params(W, bits) if row_grid is None else row_grid
         scales[:, 0], zeros[:, 0] = s, z
+    elif row_grid is not None:
+        raise ValueError("row_grid applies to per-row grids only")
     for b0 in range(0, cols, block):
         b1 = min(cols, b0 + block)
         E = np.zeros((rows, b1 - b0))

@@ -7,8 +7,10 @@ against the fp64 oracle on outputs it can compute one by one:
 * R on its trailing principal block: R[k:, k:] is the factor of the trailing block of H + lambda I
   alone (the oracle pins this), so the oracle factors just that block of the GPU's H;
 * codes and the per-row loss sum_j e_j^2 on sampled rows: rows are independent given R, and the
-  first columns of a row depend only on the leading block of R (group grids are local), so for
-  the largest layer the oracle runs the leading 1024 columns.
+  first columns of a row depend only on the leading block of R, so for the largest layer the
+  oracle runs the leading 1024 columns (group grids are local to their columns; a per-row grid
+  comes from the whole original row, so the oracle computes it from the whole row and is handed
+  it, and the GPU's per-row scales and zero points are compared with it bit for bit).
 Tolerances as in the small-size parity tests: 1e-4 relative (H entries against the scale of their
 row and column, R blocks in Frobenius norm), >= 99.5 % identical codes, loss sums within 1 %.
 """
@@ -32,7 +34,10 @@ CASES = {
     "mlp_down_4096x11008": (synth.MLP_DOWN, 12, None, 1536, None),
     "fc1_49152x12288_3bit_row": (dataclasses.replace(synth.FC1, bits=3, group=-1), 8, None, 1536,
                                  None),
+    "fc1_49152x12288_4bit_g128": (synth.FC1, 8, None, 1536, None),
     "fc2_12288x49152_4bit_g128": (synth.FC2, 16, 1024, 1024, None),
+    "fc2_12288x49152_3bit_row": (dataclasses.replace(synth.FC2, bits=3, group=-1), 16, 1024, 1024,
+                                 None),
 }
 
 
@@ -98,9 +103,15 @@ def test_full_size_against_sampled_oracle(name):
     rsel = np.sort(rng.choice(rows, n_rows, replace=False))
     ridx = torch.from_numpy(rsel).to(DEV)
     oc = cols if ocols is None else ocols
-    Wr = W[ridx][:, :oc].float().cpu().numpy()
+    Wfull = W[ridx].float().cpu().numpy()
+    Wr = Wfull[:, :oc]
     Rr = R[:oc, :oc].double().cpu().numpy()
-    ref = oracle.gptq_quantize(Wr, Rr, spec.bits, spec.group, spec.block)
+    grid = None
+    if spec.group <= 0 and oc < cols:
+        grid = oracle.quant_params(Wfull, spec.bits)
+        np.testing.assert_array_equal(scales[ridx][:, 0].cpu().numpy(), grid[0])
+        np.testing.assert_array_equal(zeros[ridx][:, 0].cpu().numpy(), grid[1].astype(np.uint8))
+    ref = oracle.gptq_quantize(Wr, Rr, spec.bits, spec.group, spec.block, row_grid=grid)
     got_codes = codes[ridx][:, :oc].cpu().numpy()
     match = (got_codes == ref["codes"]).mean()
     assert match >= 0.995, match

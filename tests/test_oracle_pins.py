@@ -239,6 +239,28 @@ def test_lazy_equals_unbatched(group, block):
     np.testing.assert_allclose(a["err"], b["err"], rtol=1e-10, atol=1e-12)
 
 
+@pytest.mark.parametrize("group,lead", [(-1, 64), (-1, 96), (32, 64)])
+def test_leading_columns_depend_only_on_leading_block(group, lead):
+    """Columns 0..k-1 of a row are quantized from R's leading k x k block alone (updates only run
+    to the right), so a run on the leading columns reproduces them -- given the grid of the whole
+    row in per-row mode (its parameters come from the original, full row)."""
+    W = _rand_W(12, 160, 42)
+    H, _ = _rand_spd(160, 43, 1.5)
+    R = oracle.inverse_hessian_factor(H)["R"]
+    full = oracle.gptq_quantize(W, R, 3, group, 32)
+    grid = oracle.quant_params(W, 3) if group <= 0 else None
+    lead_run = oracle.gptq_quantize(W[:, :lead], R[:lead, :lead], 3, group, 32, row_grid=grid)
+    for k in ("codes", "W_hat"):
+        np.testing.assert_array_equal(lead_run[k], full[k][:, :lead])
+    np.testing.assert_allclose(lead_run["err"], full["err"][:, :lead], rtol=1e-12, atol=1e-15)
+    if group <= 0:
+        # without the whole row's grid, the leading columns alone give another grid
+        alone = oracle.gptq_quantize(W[:, :lead], R[:lead, :lead], 3, group, 32)
+        assert not np.array_equal(alone["scales"], full["scales"])
+        with pytest.raises(ValueError):
+            oracle.gptq_quantize(W, R, 3, 32, 32, row_grid=grid)
+
+
 def test_loss_identity_sum_of_squared_errors():
     """(W_hat - W) H_d (W_hat - W)^T = sum_j e_j^2 per row, since W_hat - W = -e R and
     H_d = R^{-1} R^{-T} (the LDL view of the OptRot page, Definition 3.2)."""
