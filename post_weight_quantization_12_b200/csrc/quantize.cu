@@ -7,12 +7,11 @@
 // (W[:, B:] -= E R[B, B:]); the design table and the blog's "Group-wise quantization"
 // (asymmetric uniform grid per row or per group).
 //
-// Column loop layout: TPR consecutive lanes (16, or 8 for 32-column blocks) own one weight row and
-// hold the current block's values of that row in registers, four consecutive columns per lane per
-// stretch of 4 * TPR columns. The block's B x B corner of R sits in shared memory with its
-// diagonal and lower part replaced by zeros, so updates need no mask (columns at or before j are
-// left untouched). Every lane of a row computes the same codes for a sub-block of four columns
-// from values broadcast by their owner lane, so one exchange serves four columns.
+// Column loop layout: four consecutive lanes own one weight row and hold the current block's values
+// of that row in registers, four consecutive columns per lane per stretch of 16 columns. The
+// block's B x B corner of R sits in shared memory. Every lane of a row computes the same codes for
+// a sub-block of four columns from values broadcast by their owner lane, so one exchange serves
+// four columns.
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -128,67 +127,55 @@ __global__ void params_kernel(const float* __restrict__ Wh, int64_t rows, int64_
   }
 }
 
-// One block of B columns [b0, b0 + nb) for every row.
-//   group_mode: 0 = grid given per row (scales[row*G + gi_fixed]);
-//               1 = groups of `group` columns inside the block, grids computed here.
-// Lane `sub` of a row holds, in registers, the columns S*t + 4*sub + u (S = 4 TPR, t < B/S,
-// u < 4): the TPR lanes of a row together cover each S-column stretch with one float4 each, so
-// their reads of a row of R and their loads/stores of W, E and codes are contiguous segments (no
-// shared memory bank conflicts, coalesced global accesses).
-template <int B, int TPR, int THREADS>
-__global__ void __launch_bounds__(THREADS)
+// One block of B columns [b0, b0 + nb) for every row. MODE 0: the grid is given per row
+// (scales[row*G + gi_fixed]); MODE 1: groups of `group` columns (a power of two no wider than the
+// block) start inside the block, and their grids are computed here from the current weights.
+//
+// Four consecutive lanes own one row; lane `sub` holds the columns 16t + 4 sub + u (t < B/16,
+// u < 4), so the four lanes of a row cover each 16-column stretch with one float4 each and their
+// accesses to a row of R, W, E and the codes are contiguous. Columns go in sub-blocks of four,
+// 16t + 4o .. +3, owned by lane o: the four lanes take the sub-block's current values from their
+// owner, each quantizes the four columns itself (so one exchange serves four columns and nothing
+// waits for a second exchange), and then each applies the four errors to its own later columns.
+// Each weight therefore receives the updates of the earlier columns one sub-block at a time, in
+// column order, with four fused multiply-adds per sub-block in the order of its columns.
+//
+// R is not written while a layer is quantized, so the block's B x B corner of R is fetched by
+// bulk copies before the wait on the previous kernel (whose tail it overlaps). Only the entries
+// right of the diagonal are used: updates are masked to later columns instead of relying on zeros
+// below the diagonal.
+template <int B, int MODE>
+__global__ void __launch_bounds__(128)
 column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const float* __restrict__ R,
-                   int b0, int nb, int bits, int group, int group_mode, int gi_fixed,
-                   float* __restrict__ scales, uint8_t* __restrict__ zeros, int G,
-                   uint8_t* __restrict__ codes, float* __restrict__ Eb, float* __restrict__ Es,
-                   float* __restrict__ err_sq, float* __restrict__ Rb_out,
-                   float* __restrict__ Rs_out, int64_t nrest) {
-  griddep_wait();
-  griddep_launch_dependents();
-
+                   int b0, int nb, int bits, int group, int gi_fixed, float* __restrict__ scales,
+                   uint8_t* __restrict__ zeros, int G, uint8_t* __restrict__ codes,
+                   float* __restrict__ Eb, float* __restrict__ Es, float* __restrict__ err_sq,
+                   float* __restrict__ Rb_out, float* __restrict__ Rs_out, int64_t nrest,
+                   int32_t* info) {
+  constexpr int TPR = 4, THREADS = 128;
   constexpr int S = 4 * TPR;       // columns covered by one float4 from each lane of a row
   constexpr int NT = B / S;        // float4 groups per lane
   constexpr int CPL = 4 * NT;      // columns per lane
-  extern __shared__ __align__(16) float qsm[];
-  float (*Rz)[B] = reinterpret_cast<float (*)[B]>(qsm);
-  float* inv_d = qsm + B * B;
-  // the block's corner of R with its diagonal and lower part zeroed; every load in flight at once
-  // (rows are 16-byte aligned: cols % 4 == 0, b0 % 4 == 0)
-  {
-    constexpr int PER = B * B / 4 / THREADS;  // float4 per thread
-    float4 buf[PER];
-#pragma unroll
-    for (int p = 0; p < PER; ++p) {
-      const int e = threadIdx.x + p * THREADS;
-      const int i = (4 * e) / B, j = (4 * e) % B;
-      float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i < nb) {
-        const float* src = R + (b0 + i) * cols + b0 + j;
-        if (j + 3 < nb) {
-          q = *reinterpret_cast<const float4*>(src);
-        } else {
-          q.x = (j + 0 < nb) ? src[0] : 0.f;
-          q.y = (j + 1 < nb) ? src[1] : 0.f;
-          q.z = (j + 2 < nb) ? src[2] : 0.f;
-          q.w = (j + 3 < nb) ? src[3] : 0.f;
-        }
-      }
-      buf[p] = q;
-    }
-#pragma unroll
-    for (int p = 0; p < PER; ++p) {
-      const int e = threadIdx.x + p * THREADS;
-      const int i = (4 * e) / B, j = (4 * e) % B;
-      float4 q = buf[p];
-      q.x = (j + 0 > i) ? q.x : 0.f;
-      q.y = (j + 1 > i) ? q.y : 0.f;
-      q.z = (j + 2 > i) ? q.z : 0.f;
-      q.w = (j + 3 > i) ? q.w : 0.f;
-      *reinterpret_cast<float4*>(&Rz[i][j]) = q;
-    }
+  extern __shared__ __align__(128) float qsm[];
+  float* Rz = qsm;                 // [B][B]: rows b0.. of R, columns b0.. (only k > i is read)
+  float* inv_d = qsm + B * B;      // [B]: 1 / R[j][j]
+  __shared__ __align__(8) uint64_t rbar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&rbar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
   }
-  for (int i = threadIdx.x; i < B; i += blockDim.x)
-    inv_d[i] = (i < nb) ? 1.f / R[(b0 + i) * cols + b0 + i] : 0.f;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    // rows are 16-byte aligned and nb is a multiple of 4 (cols % 4 == 0, b0 % 4 == 0)
+    mbar_arrive_expect_tx(&rbar, static_cast<uint32_t>(nb) * nb * 4u);
+    for (int i = 0; i < nb; ++i)
+      bulk_load(Rz + i * B, R + (b0 + i) * cols + b0, static_cast<uint32_t>(nb) * 4u, &rbar);
+  }
+  griddep_wait();
+  griddep_launch_dependents();
+
   // the tf32 split of R[b0 : b0 + nb, b1 : cols] for the trailing product that follows this block,
   // spread over the whole grid (rows 16-byte aligned: cols % 4 == 0, b1 % 4 == 0)
   if (nrest > 0) {
@@ -219,7 +206,6 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
       }
     }
   }
-  __syncthreads();
 
   const int lane = threadIdx.x & 31;
   const int sub = lane & (TPR - 1);           // position within the row's lane group
@@ -235,17 +221,7 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   for (int t = 0; t < NT; ++t) {
     const int c = S * t + 4 * sub;
     float4 w4 = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (valid) {
-      const float* src = Wh + row * cols + b0 + c;
-      if (c + 3 < nb) {
-        w4 = *reinterpret_cast<const float4*>(src);
-      } else {
-        w4.x = (c + 0 < nb) ? src[0] : 0.f;
-        w4.y = (c + 1 < nb) ? src[1] : 0.f;
-        w4.z = (c + 2 < nb) ? src[2] : 0.f;
-        w4.w = (c + 3 < nb) ? src[3] : 0.f;
-      }
-    }
+    if (valid && c < nb) w4 = *reinterpret_cast<const float4*>(Wh + row * cols + b0 + c);
     v[4 * t + 0] = w4.x; v[4 * t + 1] = w4.y; v[4 * t + 2] = w4.z; v[4 * t + 3] = w4.w;
   }
 #pragma unroll
@@ -255,92 +231,97 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   }
   const float maxq = static_cast<float>((1 << bits) - 1);
   float s = 1.f, z = 0.f;
-  if (group_mode == 0 && valid) {
+  if (MODE == 0 && valid) {
     s = scales[row * G + gi_fixed];
     z = static_cast<float>(zeros[row * G + gi_fixed]);
   }
   float inv_s = 1.f / s;
 
-  // Columns go in sub-blocks of four, 32t + 4o .. 32t + 4o + 3, all held by lane o of the row.
-  // Every lane of the row takes the four current values from their owner and quantizes them
-  // itself, applying each column's error to the sub-block's later columns in registers; then
-  // each lane applies the four errors to its own later columns (a rank-4 update whose FMAs run in
-  // the same order as four rank-1 updates). Only the owner keeps the results.
-  int gcnt = 0;                             // position in the current group (group_mode 1)
+  // the corner of R has landed: the reciprocals of its diagonal
+  if (!mbar_wait_bounded(&rbar, 0, &abort_flag, info)) {
+    mbar_drain_bounded(&rbar, 0);            // let the copies in flight land before leaving
+    return;
+  }
+  for (int i = threadIdx.x; i < nb; i += THREADS) inv_d[i] = 1.f / Rz[i * B + i];
+  __syncthreads();
+
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
+#pragma unroll
     for (int o = 0; o < TPR; ++o) {
       const int j0 = S * t + 4 * o;
-      if (j0 >= nb) break;
+      if (j0 >= nb) break;                   // nb % 4 == 0: sub-blocks are whole
       const bool own = (sub == o);
       float w4[4], e4[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) w4[u] = __shfl_sync(0xffffffffu, v[4 * t + u], base_lane + o);
+      const float4 id4 = *reinterpret_cast<const float4*>(inv_d + j0);
+      const float idv[4] = {id4.x, id4.y, id4.z, id4.w};
+      float rin[3][4];                         // R[j0 + u][j0 .. j0 + 3], for the sub-block itself
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const float4 r4 = *reinterpret_cast<const float4*>(Rz + (j0 + u) * B + j0);
+        rin[u][0] = r4.x; rin[u][1] = r4.y; rin[u][2] = r4.z; rin[u][3] = r4.w;
+      }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int j = j0 + u;
-        e4[u] = 0.f;
-        if (j < nb) {
-          if (group_mode == 1) {
-            if (gcnt == 0) {
-              float lo = 0.f, hi = 0.f;
-              if (group <= 4) {
-                // the group lies inside this sub-block, whose current values every lane holds
+        if (MODE == 1 && (j & (group - 1)) == 0) {
+          float lo = 0.f, hi = 0.f;
+          if (group <= 4) {
+            // the group lies inside this sub-block, whose current values every lane holds
 #pragma unroll
-                for (int u2 = 0; u2 < 4; ++u2)
-                  if (u2 >= u && u2 < u + group && j0 + u2 < nb) {
-                    lo = fminf(lo, w4[u2]);
-                    hi = fmaxf(hi, w4[u2]);
-                  }
-              } else {
-                // the group starts at this sub-block (u == 0): the row's lanes hold it
-#pragma unroll
-                for (int k = 0; k < CPL; ++k) {
-                  const int c = colof(k);
-                  if (c >= j && c < j + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
-                }
-#pragma unroll
-                for (int off = TPR / 2; off > 0; off >>= 1) {
-                  lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-                  hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-                }
+            for (int u2 = 0; u2 < 4; ++u2)
+              if (u2 >= u && u2 < u + group) {
+                lo = fminf(lo, w4[u2]);
+                hi = fmaxf(hi, w4[u2]);
               }
-              grid_params(lo, hi, maxq, s, z);
-              inv_s = 1.f / s;
-              if (valid && sub == 0) {
-                const int gi = (b0 + j) / group;
-                scales[row * G + gi] = s;
-                zeros[row * G + gi] = static_cast<uint8_t>(z);
-              }
+          } else {
+            // the group starts at this sub-block (u == 0): the row's lanes hold it
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) {
+              const int c = colof(k);
+              if (c >= j && c < j + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
             }
-            gcnt = (gcnt + 1 == group) ? 0 : gcnt + 1;
-          }
-          const float w = w4[u];
-          const float q = fminf(fmaxf(rint_quot(w, s, inv_s) + z, 0.f), maxq);
-          const float wh = __fmul_rn(s, q - z);
-          const float e = __fmul_rn(__fsub_rn(w, wh), inv_d[j]);
-          e4[u] = e;
-          v[4 * t + u] = own ? wh : v[4 * t + u];
-          qf[4 * t + u] = own ? q : qf[4 * t + u];
-          err[4 * t + u] = own ? e : err[4 * t + u];
 #pragma unroll
-          for (int u2 = u + 1; u2 < 4; ++u2) w4[u2] = fmaf(-e, Rz[j][j0 + u2], w4[u2]);
+            for (int off = TPR / 2; off > 0; off >>= 1) {
+              lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+              hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
+            }
+          }
+          grid_params(lo, hi, maxq, s, z);
+          inv_s = 1.f / s;
+          if (valid && sub == 0) {
+            const int gi = (b0 + j) / group;
+            scales[row * G + gi] = s;
+            zeros[row * G + gi] = static_cast<uint8_t>(z);
+          }
         }
+        const float w = w4[u];
+        const float q = fminf(fmaxf(rint_quot(w, s, inv_s) + z, 0.f), maxq);
+        const float wh = __fmul_rn(s, q - z);
+        const float e = __fmul_rn(__fsub_rn(w, wh), idv[u]);
+        e4[u] = e;
+        v[4 * t + u] = own ? wh : v[4 * t + u];
+        qf[4 * t + u] = own ? q : qf[4 * t + u];
+        err[4 * t + u] = own ? e : err[4 * t + u];
+#pragma unroll
+        for (int u2 = u + 1; u2 < 4; ++u2) w4[u2] = fmaf(-e, rin[u][u2], w4[u2]);
       }
+      // the sub-block's errors on this lane's later columns (rank 4, one column after another)
 #pragma unroll
       for (int t2 = t; t2 < NT; ++t2) {
-        // the owner's own four columns of group t are final already
-        const bool skip = (t2 == t) && own;
+        if (t2 == t && sub <= o) continue;   // earlier columns, or the sub-block itself
         float4 r[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) r[u] = *reinterpret_cast<const float4*>(&Rz[j0 + u][S * t2 + 4 * sub]);
+        for (int u = 0; u < 4; ++u)
+          r[u] = *reinterpret_cast<const float4*>(Rz + (j0 + u) * B + S * t2 + 4 * sub);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const float c = skip ? 0.f : e4[u];
-          v[4 * t2 + 0] = fmaf(-c, r[u].x, v[4 * t2 + 0]);
-          v[4 * t2 + 1] = fmaf(-c, r[u].y, v[4 * t2 + 1]);
-          v[4 * t2 + 2] = fmaf(-c, r[u].z, v[4 * t2 + 2]);
-          v[4 * t2 + 3] = fmaf(-c, r[u].w, v[4 * t2 + 3]);
+          v[4 * t2 + 0] = fmaf(-e4[u], r[u].x, v[4 * t2 + 0]);
+          v[4 * t2 + 1] = fmaf(-e4[u], r[u].y, v[4 * t2 + 1]);
+          v[4 * t2 + 2] = fmaf(-e4[u], r[u].z, v[4 * t2 + 2]);
+          v[4 * t2 + 3] = fmaf(-e4[u], r[u].w, v[4 * t2 + 3]);
         }
       }
     }
@@ -355,34 +336,20 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
     const int c = S * t + 4 * sub;
-    float* wd = Wh + row * cols + b0 + c;
-    uint8_t* cd = codes + row * cols + b0 + c;
-    float* eb = Eb + row * B + c;
-    float* es = Es + row * B + c;
+    if (c >= nb) continue;                   // nb % 4 == 0: a float4 is whole or absent
     float b4[4], s4[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       b4[u] = tf32_rna_q(err[4 * t + u]);
       s4[u] = err[4 * t + u] - b4[u];
     }
-    if (c + 3 < nb) {
-      *reinterpret_cast<float4*>(wd) = make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
-      *reinterpret_cast<float4*>(eb) = make_float4(b4[0], b4[1], b4[2], b4[3]);
-      *reinterpret_cast<float4*>(es) = make_float4(s4[0], s4[1], s4[2], s4[3]);
-      *reinterpret_cast<uint32_t*>(cd) =
-          static_cast<uint32_t>(qf[4 * t]) | (static_cast<uint32_t>(qf[4 * t + 1]) << 8) |
-          (static_cast<uint32_t>(qf[4 * t + 2]) << 16) | (static_cast<uint32_t>(qf[4 * t + 3]) << 24);
-    } else {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (c + u < nb) {
-          wd[u] = v[4 * t + u];
-          cd[u] = static_cast<uint8_t>(qf[4 * t + u]);
-          eb[u] = b4[u];
-          es[u] = s4[u];
-        }
-      }
-    }
+    *reinterpret_cast<float4*>(Wh + row * cols + b0 + c) =
+        make_float4(v[4 * t], v[4 * t + 1], v[4 * t + 2], v[4 * t + 3]);
+    *reinterpret_cast<float4*>(Eb + row * B + c) = make_float4(b4[0], b4[1], b4[2], b4[3]);
+    *reinterpret_cast<float4*>(Es + row * B + c) = make_float4(s4[0], s4[1], s4[2], s4[3]);
+    *reinterpret_cast<uint32_t*>(codes + row * cols + b0 + c) =
+        static_cast<uint32_t>(qf[4 * t]) | (static_cast<uint32_t>(qf[4 * t + 1]) << 8) |
+        (static_cast<uint32_t>(qf[4 * t + 2]) << 16) | (static_cast<uint32_t>(qf[4 * t + 3]) << 24);
   }
   if (sub == 0 && err_sq != nullptr) err_sq[row] += sq;
 }
@@ -399,20 +366,17 @@ static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, con
                                       int nb, int bits, int group, int group_mode, int gi_fixed,
                                       float* scales, uint8_t* zeros, int G, uint8_t* codes,
                                       float* Eb, float* Es, float* err_sq, float* Rb, float* Rs,
-                                      int64_t nrest, cudaStream_t stream) {
-  // 16 lanes per row for blocks of 64 or 128 columns (more warps, less per-lane update work),
-  // 8 for 32 columns
-  constexpr int TPR = B >= 64 ? 16 : 8;
-  constexpr int THREADS = B >= 64 ? 256 : 128;
-  const int rows_per_cta = THREADS / TPR;
-  const int64_t grid = (rows + rows_per_cta - 1) / rows_per_cta;
+                                      int64_t nrest, int32_t* info, cudaStream_t stream) {
+  // four lanes per row, 32 rows per CTA
+  constexpr int THREADS = 128, ROWS_PER_CTA = 32;
+  const int64_t grid = (rows + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
   constexpr int smem = (B * B + B) * 4;
-  const gptq_status st = set_max_dynamic_smem(
-      reinterpret_cast<const void*>(column_loop_kernel<B, TPR, THREADS>), smem);
+  auto kernel = group_mode == 1 ? column_loop_kernel<B, 1> : column_loop_kernel<B, 0>;
+  const gptq_status st = set_max_dynamic_smem(reinterpret_cast<const void*>(kernel), smem);
   if (st != GPTQ_OK) return st;
-  return launch_pdl(column_loop_kernel<B, TPR, THREADS>, dim3(static_cast<unsigned>(grid)),
-                    dim3(THREADS), smem, stream, Wh, rows, cols, R, b0, nb, bits, group, group_mode,
-                    gi_fixed, scales, zeros, G, codes, Eb, Es, err_sq, Rb, Rs, nrest);
+  return launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(THREADS), smem, stream, Wh,
+                    rows, cols, R, b0, nb, bits, group, gi_fixed, scales, zeros, G, codes, Eb, Es,
+                    err_sq, Rb, Rs, nrest, info);
 }
 
 gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, int64_t cols,
@@ -468,17 +432,17 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
       case 32:
         st = launch_column_loop<32>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group, mode,
                                     gi, scales, zeros, G, codes, Eb, Es, err_sq, Rb, Rs, nrest,
-                                    stream);
+                                    info, stream);
         break;
       case 64:
         st = launch_column_loop<64>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group, mode,
                                     gi, scales, zeros, G, codes, Eb, Es, err_sq, Rb, Rs, nrest,
-                                    stream);
+                                    info, stream);
         break;
       default:
         st = launch_column_loop<128>(Wh, rows, cols, R, static_cast<int>(b0), nb, bits, group,
                                      mode, gi, scales, zeros, G, codes, Eb, Es, err_sq, Rb, Rs,
-                                     nrest, stream);
+                                     nrest, info, stream);
         break;
     }
     if (st != GPTQ_OK) return st;
