@@ -52,9 +52,36 @@ __device__ __forceinline__ void decode_lower(int st, int& I, int& J) {
   J = st - i * (i + 1) / 2;
 }
 
+// The order in which the pairs take super-tiles. The pairs of one round (consecutive super-tiles)
+// stream the same token slab at about the same time, so what HBM delivers per round is the
+// channel blocks their super-tiles touch. Row-major order over the lower triangle gives a round
+// one block row and ~n_pairs block columns (~75 distinct blocks at 49152 channels); here the
+// triangle is cut into panels of kPanel block rows, taken block column by block column, so a round
+// spans about kPanel rows and n_pairs / kPanel columns (~18 distinct blocks).
+constexpr int kPanel = 8;
+__device__ __forceinline__ void decode_panel(int st, int T, int& I, int& J) {
+  int p = 0;
+  while ((p + 1) * kPanel < T && ((p + 1) * kPanel) * ((p + 1) * kPanel + 1) / 2 <= st) ++p;
+  const int r0 = p * kPanel, h = min(kPanel, T - r0);
+  int idx = st - r0 * (r0 + 1) / 2;
+  if (idx < r0 * h) {                       // block columns left of the panel: full height
+    I = r0 + idx % h;
+    J = idx / h;
+    return;
+  }
+  idx -= r0 * h;                            // the panel's own triangle, column by column
+  int q = 0;
+  while (idx >= h - q) {
+    idx -= h - q;
+    ++q;
+  }
+  I = r0 + q + idx;
+  J = r0 + q;
+}
+
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(syrk::kThreads, 1)
 hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict__ S, int cols,
-                     int n_kblocks, int n_super, int32_t* info) {
+                     int n_kblocks, int n_super, int n_s, int32_t* info) {
   using namespace syrk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -105,7 +132,7 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
       long long issued = 0;
       for (int st = pair; st < n_super && !abort_flag; st += n_pairs) {
         int I, J;
-        decode_lower(st, I, J);
+        decode_panel(st, n_s, I, J);
         const bool diag = (I == J);
         const uint32_t bytes = diag ? kHalfBytes : kStageBytes;   // this CTA's share
         for (int kb = 0; kb < n_kblocks; ++kb) {
@@ -143,7 +170,7 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
       int chunk = 0;
       for (int st = pair; st < n_super && !abort_flag; st += n_pairs) {
         int I, J;
-        decode_lower(st, I, J);
+        decode_panel(st, n_s, I, J);
         const bool diag = (I == J);
         for (int kc = 0; kc < n_kblocks; kc += kChunkStages, ++chunk) {
           const int buf = chunk & 1;
@@ -183,7 +210,7 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
     bool ok = true;
     for (int st = pair; st < n_super && ok && !abort_flag; st += n_pairs) {
       int I, J;
-      decode_lower(st, I, J);
+      decode_panel(st, n_s, I, J);
       float acc[128];
 #pragma unroll
       for (int j = 0; j < 128; ++j) acc[j] = 0.f;
@@ -311,7 +338,7 @@ gptq_status launch_hessian_bf16(float* S, int64_t cols, const void* X, int64_t n
   const int max_pairs = num_sms() / 2;
   const int pairs = n_super < max_pairs ? n_super : max_pairs;
   hessian_syrk_bf16_tc<<<2 * pairs, kThreads, kSmemBytes, stream>>>(
-      tmap, S, static_cast<int>(cols), static_cast<int>(n_kb), n_super, info);
+      tmap, S, static_cast<int>(cols), static_cast<int>(n_kb), n_super, n_s, info);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }

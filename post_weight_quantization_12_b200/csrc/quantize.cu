@@ -7,8 +7,8 @@
 // (W[:, B:] -= E R[B, B:]); the design table and the blog's "Group-wise quantization"
 // (asymmetric uniform grid per row or per group).
 //
-// Column loop layout: four consecutive lanes own one weight row and hold the current block's values
-// of that row in registers, four consecutive columns per lane per stretch of 16 columns. The
+// Column loop layout: eight consecutive lanes own one weight row and hold the current block's values
+// of that row in registers, four consecutive columns per lane per stretch of 32 columns. The
 // block's B x B corner of R sits in shared memory. Every lane of a row computes the same codes for
 // a sub-block of four columns from values broadcast by their owner lane, so one exchange serves
 // four columns.
@@ -54,6 +54,62 @@ __device__ __forceinline__ float rint_quot(float w, float s, float inv_s) {
   // |y - r| < 0.5 - 1e-5 (|y| + 1): a margin at least as wide as 1e-5 max(1, |y|)
   if (fabsf(y - r) < fmaf(-1e-5f, fabsf(y), 0.5f - 1e-5f)) return r;
   return rintf(__fdiv_rn(w, s));
+}
+
+// Quantizes the four columns of a sub-block in order: w4 holds their current values, rin[u][u2]
+// = R[j0 + u][j0 + u2] (u2 > u) and idv[u] = 1 / R[j0 + u][j0 + u]. Each column's error is applied
+// to the sub-block's later columns before they are quantized. Outputs, per column: the rounded
+// quotient clamped to the grid (rc = q - z), the zero point z it used, the dequantized value and
+// the error; and, in group mode, the grid of each column that starts a group of one or two
+// columns (gs, gz).
+// FAST: rint(w * (1/s)) with no branch; returns true if some quotient lies too near a half-integer
+// for that product to decide its rounding -- the caller then redoes the sub-block with FAST =
+// false, where rint_quot decides such columns by the correctly rounded division.
+template <bool FAST, int MODE>
+__device__ __forceinline__ bool quantize_sub_block(float (&w4)[4], const float (&rin)[3][4],
+                                                   const float (&idv)[4], float& s, float& z,
+                                                   float& inv_s, float maxq, int group, int j0,
+                                                   float (&rc4)[4], float (&zq)[4],
+                                                   float (&wh4)[4], float (&e4)[4],
+                                                   float (&gs)[4], float (&gz)[4]) {
+  bool near = false;
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    if (MODE == 1 && group < 4 && ((j0 + u) & (group - 1)) == 0) {
+      // a group of one or two columns starts here: its current values are in w4
+      float lo = 0.f, hi = 0.f;
+#pragma unroll
+      for (int u2 = 0; u2 < 4; ++u2)
+        if (u2 >= u && u2 < u + group) {
+          lo = fminf(lo, w4[u2]);
+          hi = fmaxf(hi, w4[u2]);
+        }
+      grid_params(lo, hi, maxq, s, z);
+      inv_s = 1.f / s;
+      gs[u] = s;
+      gz[u] = z;
+    }
+    const float w = w4[u];
+    float r;
+    if (FAST) {
+      const float y = w * inv_s;
+      r = rintf(y);
+      near |= !(fabsf(y - r) < fmaf(-1e-5f, fabsf(y), 0.5f - 1e-5f));
+    } else {
+      r = rint_quot(w, s, inv_s);
+    }
+    // clamp(r + z, 0, maxq) - z, exactly (small integers)
+    const float rc = fminf(fmaxf(r, -z), maxq - z);
+    const float wh = __fmul_rn(s, rc);
+    const float e = __fmul_rn(__fsub_rn(w, wh), idv[u]);
+    rc4[u] = rc;
+    zq[u] = z;
+    wh4[u] = wh;
+    e4[u] = e;
+#pragma unroll
+    for (int u2 = u + 1; u2 < 4; ++u2) w4[u2] = fmaf(-e, rin[u][u2], w4[u2]);
+  }
+  return near;
 }
 
 template <typename T>
@@ -131,10 +187,10 @@ __global__ void params_kernel(const float* __restrict__ Wh, int64_t rows, int64_
 // (scales[row*G + gi_fixed]); MODE 1: groups of `group` columns (a power of two no wider than the
 // block) start inside the block, and their grids are computed here from the current weights.
 //
-// Four consecutive lanes own one row; lane `sub` holds the columns 16t + 4 sub + u (t < B/16,
-// u < 4), so the four lanes of a row cover each 16-column stretch with one float4 each and their
+// TPR consecutive lanes own one row; lane `sub` holds the columns S t + 4 sub + u (S = 4 TPR,
+// t < B/S, u < 4), so the lanes of a row cover each S-column stretch with one float4 each and their
 // accesses to a row of R, W, E and the codes are contiguous. Columns go in sub-blocks of four,
-// 16t + 4o .. +3, owned by lane o: the four lanes take the sub-block's current values from their
+// S t + 4o .. +3, owned by lane o: the row's lanes take the sub-block's current values from their
 // owner, each quantizes the four columns itself (so one exchange serves four columns and nothing
 // waits for a second exchange), and then each applies the four errors to its own later columns.
 // Each weight therefore receives the updates of the earlier columns one sub-block at a time, in
@@ -144,7 +200,7 @@ __global__ void params_kernel(const float* __restrict__ Wh, int64_t rows, int64_
 // bulk copies before the wait on the previous kernel (whose tail it overlaps). Only the entries
 // right of the diagonal are used: updates are masked to later columns instead of relying on zeros
 // below the diagonal.
-template <int B, int MODE>
+template <int B, int MODE, int TPR>
 __global__ void __launch_bounds__(128)
 column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const float* __restrict__ R,
                    int b0, int nb, int bits, int group, int gi_fixed, float* __restrict__ scales,
@@ -152,7 +208,7 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
                    float* __restrict__ Eb, float* __restrict__ Es, float* __restrict__ err_sq,
                    float* __restrict__ Rb_out, float* __restrict__ Rs_out, int64_t nrest,
                    int32_t* info) {
-  constexpr int TPR = 4, THREADS = 128;
+  constexpr int THREADS = 128;
   constexpr int S = 4 * TPR;       // columns covered by one float4 from each lane of a row
   constexpr int NT = B / S;        // float4 groups per lane
   constexpr int CPL = 4 * NT;      // columns per lane
@@ -212,6 +268,7 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   const int base_lane = lane & ~(TPR - 1);
   const int64_t row = blockIdx.x * static_cast<int64_t>(THREADS / TPR) + threadIdx.x / TPR;
   const bool valid = row < rows;
+
   auto colof = [&](int k) { return S * (k >> 2) + 4 * sub + (k & 3); };  // block column of v[k]
 
   float v[CPL];
@@ -245,9 +302,11 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
   for (int i = threadIdx.x; i < nb; i += THREADS) inv_d[i] = 1.f / Rz[i * B + i];
   __syncthreads();
 
+  // The stretch index t is unrolled (register indices must be constants); the sub-blocks of a
+  // stretch run as a loop, which keeps the kernel small enough for the instruction cache.
 #pragma unroll
   for (int t = 0; t < NT; ++t) {
-#pragma unroll
+#pragma unroll 1
     for (int o = 0; o < TPR; ++o) {
       const int j0 = S * t + 4 * o;
       if (j0 >= nb) break;                   // nb % 4 == 0: sub-blocks are whole
@@ -263,50 +322,64 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
         const float4 r4 = *reinterpret_cast<const float4*>(Rz + (j0 + u) * B + j0);
         rin[u][0] = r4.x; rin[u][1] = r4.y; rin[u][2] = r4.z; rin[u][3] = r4.w;
       }
+      if (MODE == 1 && group >= 4 && (j0 & (group - 1)) == 0) {
+        // a group of four or more columns starts here (at the sub-block's first column)
+        float lo = 0.f, hi = 0.f;
+        if (group == 4) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = j0 + u;
-        if (MODE == 1 && (j & (group - 1)) == 0) {
-          float lo = 0.f, hi = 0.f;
-          if (group <= 4) {
-            // the group lies inside this sub-block, whose current values every lane holds
-#pragma unroll
-            for (int u2 = 0; u2 < 4; ++u2)
-              if (u2 >= u && u2 < u + group) {
-                lo = fminf(lo, w4[u2]);
-                hi = fmaxf(hi, w4[u2]);
-              }
-          } else {
-            // the group starts at this sub-block (u == 0): the row's lanes hold it
-#pragma unroll
-            for (int k = 0; k < CPL; ++k) {
-              const int c = colof(k);
-              if (c >= j && c < j + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
-            }
-#pragma unroll
-            for (int off = TPR / 2; off > 0; off >>= 1) {
-              lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
-              hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
-            }
+          for (int u2 = 0; u2 < 4; ++u2) {
+            lo = fminf(lo, w4[u2]);
+            hi = fmaxf(hi, w4[u2]);
           }
-          grid_params(lo, hi, maxq, s, z);
-          inv_s = 1.f / s;
-          if (valid && sub == 0) {
-            const int gi = (b0 + j) / group;
-            scales[row * G + gi] = s;
-            zeros[row * G + gi] = static_cast<uint8_t>(z);
+        } else {
+          // the row's lanes hold it
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            const int c = colof(k);
+            if (c >= j0 && c < j0 + group && c < nb) { lo = fminf(lo, v[k]); hi = fmaxf(hi, v[k]); }
+          }
+#pragma unroll
+          for (int off = TPR / 2; off > 0; off >>= 1) {
+            lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, off));
+            hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, off));
           }
         }
-        const float w = w4[u];
-        const float q = fminf(fmaxf(rint_quot(w, s, inv_s) + z, 0.f), maxq);
-        const float wh = __fmul_rn(s, q - z);
-        const float e = __fmul_rn(__fsub_rn(w, wh), idv[u]);
-        e4[u] = e;
-        v[4 * t + u] = own ? wh : v[4 * t + u];
-        qf[4 * t + u] = own ? q : qf[4 * t + u];
-        err[4 * t + u] = own ? e : err[4 * t + u];
+        grid_params(lo, hi, maxq, s, z);
+        inv_s = 1.f / s;
+        if (valid && sub == 0) {
+          const int gi = (b0 + j0) / group;
+          scales[row * G + gi] = s;
+          zeros[row * G + gi] = static_cast<uint8_t>(z);
+        }
+      }
+      // the four columns, first with the branch-free rounding; if any quotient of the warp lies
+      // near a half-integer, again from the same inputs with the exact decision
+      float rc4[4], zq[4], wh4[4], gs[4], gz[4];
+      {
+        float w_in[4] = {w4[0], w4[1], w4[2], w4[3]};
+        const float s0 = s, z0 = z, is0 = inv_s;
+        const bool near = quantize_sub_block<true, MODE>(w4, rin, idv, s, z, inv_s, maxq, group,
+                                                         j0, rc4, zq, wh4, e4, gs, gz);
+        if (__any_sync(0xffffffffu, near)) {
+          s = s0; z = z0; inv_s = is0;
+          quantize_sub_block<false, MODE>(w_in, rin, idv, s, z, inv_s, maxq, group, j0, rc4, zq,
+                                          wh4, e4, gs, gz);
+        }
+      }
+      if (MODE == 1 && group < 4 && valid && sub == 0) {
 #pragma unroll
-        for (int u2 = u + 1; u2 < 4; ++u2) w4[u2] = fmaf(-e, rin[u][u2], w4[u2]);
+        for (int u = 0; u < 4; ++u)
+          if (((j0 + u) & (group - 1)) == 0) {
+            const int gi = (b0 + j0 + u) / group;
+            scales[row * G + gi] = gs[u];
+            zeros[row * G + gi] = static_cast<uint8_t>(gz[u]);
+          }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v[4 * t + u] = own ? wh4[u] : v[4 * t + u];
+        qf[4 * t + u] = own ? rc4[u] + zq[u] : qf[4 * t + u];
+        err[4 * t + u] = own ? e4[u] : err[4 * t + u];
       }
       // the sub-block's errors on this lane's later columns (rank 4, one column after another)
 #pragma unroll
@@ -367,11 +440,11 @@ static gptq_status launch_column_loop(float* Wh, int64_t rows, int64_t cols, con
                                       float* scales, uint8_t* zeros, int G, uint8_t* codes,
                                       float* Eb, float* Es, float* err_sq, float* Rb, float* Rs,
                                       int64_t nrest, int32_t* info, cudaStream_t stream) {
-  // four lanes per row, 32 rows per CTA
-  constexpr int THREADS = 128, ROWS_PER_CTA = 32;
+  // TPR lanes per row, 128 / TPR rows per CTA
+  constexpr int TPR = 8, THREADS = 128, ROWS_PER_CTA = THREADS / TPR;
   const int64_t grid = (rows + ROWS_PER_CTA - 1) / ROWS_PER_CTA;
   constexpr int smem = (B * B + B) * 4;
-  auto kernel = group_mode == 1 ? column_loop_kernel<B, 1> : column_loop_kernel<B, 0>;
+  auto kernel = group_mode == 1 ? column_loop_kernel<B, 1, TPR> : column_loop_kernel<B, 0, TPR>;
   const gptq_status st = set_max_dynamic_smem(reinterpret_cast<const void*>(kernel), smem);
   if (st != GPTQ_OK) return st;
   return launch_pdl(kernel, dim3(static_cast<unsigned>(grid)), dim3(THREADS), smem, stream, Wh,
