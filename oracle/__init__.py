@@ -6,6 +6,7 @@ from .gptq_oracle import (  # noqa: F401
 )
 from .w4a16 import (  # noqa: F401
     pack_codes, unpack_codes, dequantize, w4a16_matmul, w4a16_abs_terms, group_of_column,
+    pack_codes_3bit, unpack_codes_3bit,
 )
 from .rotation import (  # noqa: F401
     hadamard_block, rotation_matrix, rotate, rotate_abs_terms, weight_incoherence,

@@ -22,6 +22,10 @@ Readings taken where the pages are silent:
     n activation vectors of length cols (token-major, like the calibration input), Y is n x rows.
   * Precision: the activations are BF16 values; the oracle forms s * (q - z) * x exactly in fp64
     and sums in fp64.
+  * Packed 3-bit layout (for the 3-bit grids; the pages fix none either): 32 codes per three
+    little-endian 32-bit words, row by row; the 32 codes of columns 32k .. 32k + 31 form the
+    96-bit little-endian number sum_i q_i 8^i held in words (r, 3k), (r, 3k + 1), (r, 3k + 2), so
+    code i sits in bits 3i .. 3i + 2 of that number (codes 10 and 21 straddle two words).
 """
 from __future__ import annotations
 
@@ -55,6 +59,43 @@ def unpack_codes(words: np.ndarray) -> np.ndarray:
     for p in range(CODES_PER_WORD):
         out[:, :, p] = (words >> np.uint32(BITS * p)) & np.uint32(0xF)
     return out.reshape(rows, nw * CODES_PER_WORD)
+
+
+def pack_codes_3bit(codes: np.ndarray) -> np.ndarray:
+    """uint8 codes [rows, cols] (values < 8, cols % 32 == 0) -> uint32 words [rows, 3 cols / 32]
+    in the 3-bit layout stated in the module header: each group of 32 codes is written out as the
+    base-8 digits of one 96-bit number, least significant first."""
+    codes = np.asarray(codes)
+    rows, cols = codes.shape
+    if cols % 32:
+        raise ValueError("cols must be a multiple of 32")
+    if codes.size and int(codes.max()) >= 8:
+        raise ValueError("codes must fit in 3 bits")
+    words = np.zeros((rows, 3 * cols // 32), np.uint32)
+    for r in range(rows):
+        for k in range(cols // 32):
+            value = 0
+            for i in range(32):
+                value += int(codes[r, 32 * k + i]) << (3 * i)
+            for j in range(3):
+                words[r, 3 * k + j] = (value >> (32 * j)) & 0xFFFFFFFF
+    return words
+
+
+def unpack_codes_3bit(words: np.ndarray) -> np.ndarray:
+    """Inverse of pack_codes_3bit: uint32 [rows, 3 cols / 32] -> uint8 [rows, cols]."""
+    words = np.asarray(words, dtype=np.uint32)
+    rows, nw = words.shape
+    if nw % 3:
+        raise ValueError("a row holds whole groups of three words")
+    out = np.zeros((rows, nw // 3 * 32), np.uint8)
+    for r in range(rows):
+        for k in range(nw // 3):
+            value = (int(words[r, 3 * k]) | (int(words[r, 3 * k + 1]) << 32) |
+                     (int(words[r, 3 * k + 2]) << 64))
+            for i in range(32):
+                out[r, 32 * k + i] = (value >> (3 * i)) & 7
+    return out
 
 
 def group_of_column(cols: int, group: int) -> np.ndarray:

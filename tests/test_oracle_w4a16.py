@@ -123,3 +123,56 @@ def test_matmul_linear_in_x_and_zero_point():
     assert np.allclose(f(codes, zeros, X1 + 2 * X2), f(codes, zeros, X1) + 2 * f(codes, zeros, X2),
                        rtol=1e-13, atol=1e-15)
     assert np.allclose(f(codes + 3, zeros + 3, X1), f(codes, zeros, X1), rtol=1e-14, atol=1e-16)
+
+
+# ---------------------------------------------------------------------------------------------
+# Packed 3-bit layout (32 codes per three words)
+# ---------------------------------------------------------------------------------------------
+
+def _codes3(rows, cols, seed):
+    return np.random.default_rng(seed).integers(0, 8, (rows, cols), dtype=np.uint8)
+
+
+def test_pack3_layout_is_little_endian_base8():
+    """Each group of 32 codes, read as an octal numeral with column 32k as its last digit (the
+    least significant), is the 96-bit number held in the group's three words, word 3k lowest.
+    The numeral is converted by Python's own base-8 parser, not by shifts."""
+    codes = _codes3(4, 96, 11)
+    words = oracle.pack_codes_3bit(codes)
+    assert words.dtype == np.uint32 and words.shape == (4, 9)
+    for r in range(4):
+        for k in range(3):
+            numeral = "".join(str(int(d)) for d in codes[r, 32 * k:32 * k + 32][::-1])
+            value = int(numeral, 8)
+            got = int(words[r, 3 * k]) + (int(words[r, 3 * k + 1]) << 32) + \
+                (int(words[r, 3 * k + 2]) << 64)
+            assert got == value
+
+
+@pytest.mark.parametrize("col,expect", [
+    (0, (0x7, 0, 0)),                    # bits 0..2
+    (10, (0xC0000000, 0x1, 0)),          # bits 30..32: straddles words 0 and 1
+    (11, (0, 0xE, 0)),                   # bits 33..35
+    (21, (0, 0x80000000, 0x3)),          # bits 63..65: straddles words 1 and 2
+    (31, (0, 0, 0xE0000000)),            # bits 93..95
+])
+def test_pack3_single_code_probe(col, expect):
+    """One code of 7 (all three bits set) in an otherwise zero group: the set bits, worked out by
+    hand from the bit offsets 3 col .. 3 col + 2, land exactly in the words given."""
+    codes = np.zeros((1, 32), np.uint8)
+    codes[0, col] = 7
+    assert tuple(int(w) for w in oracle.pack_codes_3bit(codes)[0]) == expect
+
+
+def test_pack3_round_trip_and_rejects():
+    codes = _codes3(5, 128, 12)
+    assert np.array_equal(oracle.unpack_codes_3bit(oracle.pack_codes_3bit(codes)), codes)
+    with pytest.raises(ValueError):
+        oracle.pack_codes_3bit(codes[:, :96 + 16])
+    bad = codes.copy()
+    bad[2, 5] = 8
+    with pytest.raises(ValueError):
+        oracle.pack_codes_3bit(bad)
+    # the 3-bit form of codes that fit in 3 bits holds the same values as the 4-bit form
+    assert np.array_equal(oracle.unpack_codes(oracle.pack_codes(codes)),
+                          oracle.unpack_codes_3bit(oracle.pack_codes_3bit(codes)))
