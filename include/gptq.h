@@ -64,7 +64,7 @@ typedef enum gptq_route {
  *                   step route only). */
 #define GPTQ_INFO_TIMEOUT (-1)        /* a bounded wait inside a kernel expired */
 #define GPTQ_INFO_BAD_HESSIAN (-2)    /* mean(diag H) <= 0 or not finite: nothing to damp */
-#define GPTQ_INFO_BAD_CODE (-3)       /* gptq_pack_codes_4bit met a code >= 16 */
+#define GPTQ_INFO_BAD_CODE (-3)       /* a pack call met a code too wide for its format */
 
 /* Which workspace gptq_workspace_size() reports. */
 #define GPTQ_WS_PREPARE 1
@@ -238,13 +238,40 @@ gptq_status gptq_pack_codes_4bit(const uint8_t* codes_dev, int64_t rows, int64_t
                                  uint32_t* packed_dev, int32_t* info_dev, void* stream);
 
 /*
+ * Packed 3-bit codes -- the storage for layers quantized on 3-bit grids (8 levels), 3/8 of the
+ * uint8 code bytes.
+ *
+ * Source: as gptq_pack_codes_4bit ("GPTQ second-order quantization" blog, "What the original
+ * results established"; the Vietnamese version, "Group-wise quantization"): the packed layout is
+ * chosen with the bit width and the runtime kernel, and the pages fix none. This one is:
+ *   32 codes per three little-endian 32-bit words, row after row: the codes of columns 32k ..
+ *   32k + 31 of row r form the 96-bit little-endian number sum_i q_i 8^i held in words
+ *   packed[r * (3 * cols / 32) + 3k + j], j = 0, 1, 2 (word j holding bits 32j .. 32j + 31);
+ *   code (r, c) therefore sits in bits 3 (c % 32) .. 3 (c % 32) + 2, and the codes of columns
+ *   32k + 10 and 32k + 21 straddle two words.
+ *
+ *   codes_dev   uint8 [rows x ldc] (columns 0..cols-1 used), e.g. gptq_quantize_layer's codes at
+ *               bits <= 3. 8-byte aligned, ldc % 8 == 0.
+ *   packed_dev  uint32 [rows x 3 cols/32], dense (row stride 3 cols / 8 bytes), 4-byte aligned;
+ *               written.
+ *   info_dev    status word (may be NULL): GPTQ_INFO_BAD_CODE if a code is 8 or more; its low
+ *               three bits are stored.
+ * rows == 0 enqueues nothing. Errors: GPTQ_EINVAL (null pointers, cols <= 0, cols % 32 != 0,
+ * ldc < cols, ldc % 8 != 0, alignment).
+ */
+gptq_status gptq_pack_codes_3bit(const uint8_t* codes_dev, int64_t rows, int64_t cols, int64_t ldc,
+                                 uint32_t* packed_dev, int32_t* info_dev, void* stream);
+
+/*
  * W4A16 product: Y = X W_hat^T with W_hat read from packed 4-bit codes and dequantized on the fly,
  *   Y[n][r] = sum_c X[n][c] * s[r, g(c)] * (q[r][c] - z[r, g(c)]),  g(c) = c / group (0 per row).
  *
  * Source: "GPTQ second-order quantization" blog, "What the original results established" (W4A16:
  * BF16 activations, weight bytes moved packed and dequantized in the kernel) and "Group-wise
  * quantization" (scale and zero point per row or per group of input channels). One call serves a
- * decode step (n = 1, a matrix-vector product) or a small batch of activation vectors (n <= 16).
+ * decode step (n = 1, a matrix-vector product), a small batch of activation vectors (n <= 16, the
+ * same kernel) or a larger batch (n > 16: a tensor-core kernel, weights as the MMA's 128-row M,
+ * activation rows as its N).
  *
  *   packed_dev  codes in the layout of gptq_pack_codes_4bit, [rows x cols/8] uint32, 16-byte
  *               aligned.
@@ -259,10 +286,12 @@ gptq_status gptq_pack_codes_4bit(const uint8_t* codes_dev, int64_t rows, int64_t
  * Empty calls (rows == 0 or n == 0) are checked for shapes only and may pass NULL buffers.
  * Arithmetic: q - z is formed exactly in bf16 and multiplied by X on the tensor cores with fp32
  * accumulation over each 128-column chunk; the chunk sum is scaled by s in fp32 and the chunks
- * are added in a fixed order, so results are deterministic for a given device and shape.
+ * are added in a fixed order, so results are deterministic for a given device and shape. For
+ * n > 16 on a layer with few 128-row tiles the columns may be split in two halves whose sums are
+ * added into Y after Y is zeroed (a sum of two terms onto zero does not depend on their order).
  * rows == 0 or n == 0 enqueues nothing. Errors: GPTQ_EINVAL (null pointers, cols <= 0,
  * cols % 32 != 0, group rules, ld or alignment rules, n < 0), GPTQ_EUNSUPPORTED (x_dtype other than
- * GPTQ_BF16, n > 16, rows above 2^27, cols above 2^22, rows * G of 2^31 or more).
+ * GPTQ_BF16, n above 65535 * 128, rows above 2^27, cols above 2^22, rows * G of 2^31 or more).
  */
 gptq_status gptq_w4a16_matmul(const uint32_t* packed_dev, const float* scales_dev,
                               const uint8_t* zeros_dev, int64_t rows, int64_t cols, int group,

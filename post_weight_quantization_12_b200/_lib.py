@@ -39,6 +39,7 @@ SIGNATURES = {
                                            _P, _P, _P, _P, _P, _P]),
     "gptq_kernel_launches": (ctypes.c_uint64, []),
     "gptq_pack_codes_4bit": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P]),
+    "gptq_pack_codes_3bit": (_I32, [_P, _I64, _I64, _I64, _P, _P, _P]),
     "gptq_hadamard_block": (_I32, [_I64]),
     "gptq_obq_quantize": (_I32, [_P, _I64, _I64, _I64, _P, _I32, _I32, _P, _P, _P, _P, _P, _P,
                                  _P]),
@@ -185,6 +186,19 @@ def pack_codes_4bit(codes, packed, info=None, stream=None):
     st = load().gptq_pack_codes_4bit(_ptr(codes), codes.shape[0], 8 * packed.shape[1], ldc,
                                      _ptr(packed), _ptr(info), _stream(stream))
     _check(st, "gptq_pack_codes_4bit")
+
+
+def pack_codes_3bit(codes, packed, info=None, stream=None):
+    """uint8 codes[rows, >= cols] (values < 8) -> packed[rows, 3 cols // 32] (int32 or uint32
+    tensor, the 32-bit words of the 3-bit layout in include/gptq.h); cols = 32 * packed.shape[1]
+    // 3."""
+    ldc = _row_major_ld(codes, "codes")
+    if packed.dim() != 2 or not packed.is_contiguous() or packed.element_size() != 4 or \
+            packed.shape[1] % 3:
+        raise ValueError("packed must be a contiguous 2-D tensor of 32-bit words, 3 per 32 codes")
+    st = load().gptq_pack_codes_3bit(_ptr(codes), codes.shape[0], 32 * (packed.shape[1] // 3),
+                                     ldc, _ptr(packed), _ptr(info), _stream(stream))
+    _check(st, "gptq_pack_codes_3bit")
 
 
 def w4a16_matmul(packed, scales, zeros, group, X, Y, info=None, stream=None):

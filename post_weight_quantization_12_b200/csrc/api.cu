@@ -191,6 +191,16 @@ gptq_status gptq_pack_codes_4bit(const uint8_t* codes_dev, int64_t rows, int64_t
                              static_cast<cudaStream_t>(stream));
 }
 
+gptq_status gptq_pack_codes_3bit(const uint8_t* codes_dev, int64_t rows, int64_t cols, int64_t ldc,
+                                 uint32_t* packed_dev, int32_t* info_dev, void* stream) {
+  if (rows < 0 || cols <= 0 || cols % 32 != 0 || ldc < cols || ldc % 8 != 0) return GPTQ_EINVAL;
+  if (rows == 0) return GPTQ_OK;  // empty: the buffers may be absent
+  if (codes_dev == nullptr || packed_dev == nullptr) return GPTQ_EINVAL;
+  if (!aligned(codes_dev, 8) || !aligned(packed_dev, 4)) return GPTQ_EINVAL;
+  return run_pack_codes_3bit(codes_dev, rows, cols, ldc, packed_dev, info_dev,
+                             static_cast<cudaStream_t>(stream));
+}
+
 gptq_status gptq_w4a16_matmul(const uint32_t* packed_dev, const float* scales_dev,
                               const uint8_t* zeros_dev, int64_t rows, int64_t cols, int group,
                               const void* X_dev, gptq_dtype x_dtype, int64_t n, int64_t ldx,
@@ -199,7 +209,7 @@ gptq_status gptq_w4a16_matmul(const uint32_t* packed_dev, const float* scales_de
   if (group != -1 && (group <= 0 || group % 128 != 0 || cols % group != 0)) return GPTQ_EINVAL;
   if (ldx < cols || ldx % 8 != 0 || ldy < rows) return GPTQ_EINVAL;
   if (x_dtype != GPTQ_BF16) return x_dtype == GPTQ_FP32 ? GPTQ_EUNSUPPORTED : GPTQ_EINVAL;
-  if (n > 16) return GPTQ_EUNSUPPORTED;
+  if (n > (static_cast<int64_t>(65535) * 128)) return GPTQ_EUNSUPPORTED;
   if (rows > (static_cast<int64_t>(1) << 27) || cols > (static_cast<int64_t>(1) << 22) ||
       rows * (group > 0 ? cols / group : 1) >= (static_cast<int64_t>(1) << 31))
     return GPTQ_EUNSUPPORTED;
@@ -208,6 +218,9 @@ gptq_status gptq_w4a16_matmul(const uint32_t* packed_dev, const float* scales_de
       Y_dev == nullptr)
     return GPTQ_EINVAL;
   if (!aligned(packed_dev, 16) || !aligned(X_dev, 16)) return GPTQ_EINVAL;
+  if (n > 16)
+    return run_w4a16_gemm(packed_dev, scales_dev, zeros_dev, rows, cols, group, X_dev, n, ldx,
+                          Y_dev, ldy, info_dev, static_cast<cudaStream_t>(stream));
   return run_w4a16_gemv(packed_dev, scales_dev, zeros_dev, rows, cols, group, X_dev, n, ldx, Y_dev,
                         ldy, info_dev, static_cast<cudaStream_t>(stream));
 }

@@ -84,6 +84,12 @@ gptq_status run_quantize_layer(const void* W, gptq_dtype w_dtype, int64_t rows, 
 // Packed 4-bit codes and the W4A16 product (w4a16.cu).
 gptq_status run_pack_codes_4bit(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ldc,
                                 uint32_t* packed, int32_t* info, cudaStream_t stream);
+gptq_status run_pack_codes_3bit(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ldc,
+                                uint32_t* packed, int32_t* info, cudaStream_t stream);
+// n > 16 activation rows: the tensor-core form of the same product (w4a16_gemm.cu).
+gptq_status run_w4a16_gemm(const uint32_t* packed, const float* scales, const uint8_t* zeros,
+                           int64_t rows, int64_t cols, int group, const void* x, int64_t n,
+                           int64_t ldx, float* y, int64_t ldy, int32_t* info, cudaStream_t stream);
 gptq_status run_w4a16_gemv(const uint32_t* packed, const float* scales, const uint8_t* zeros,
                            int64_t rows, int64_t cols, int group, const void* x, int64_t n,
                            int64_t ldx, float* y, int64_t ldy, int32_t* info, cudaStream_t stream);

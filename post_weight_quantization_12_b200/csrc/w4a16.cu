@@ -10,11 +10,15 @@
 // products).
 //
 // Layout of the packed codes: eight codes per little-endian 32-bit word, row after row; code
-// (r, c) sits in bits 4 (c mod 8) .. 4 (c mod 8) + 3 of word (r, c div 8).
+// (r, c) sits in bits 4 (c mod 8) .. 4 (c mod 8) + 3 of word (r, c div 8). Packed 3-bit codes (for
+// 3-bit grids): 32 codes per three words, the group's codes forming one 96-bit little-endian
+// number, code (r, c) in its bits 3 (c mod 32) .. 3 (c mod 32) + 2; the group of columns 32k ..
+// 32k + 31 of row r is words 3k .. 3k + 2 of the row.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <mutex>
 
 #include "common.cuh"
@@ -45,6 +49,44 @@ pack_codes_4bit_kernel(const uint8_t* __restrict__ codes, int64_t rows, int64_t 
     const uint32_t even = __byte_perm(a, b, 0x6420);  // codes 0, 2, 4, 6
     const uint32_t odd = __byte_perm(a, b, 0x7531);   // codes 1, 3, 5, 7
     packed[k] = even | (odd << 4);
+  }
+  if (bad) record_info(info, GPTQ_INFO_BAD_CODE);
+  griddep_launch_dependents();
+}
+
+// Eight 3-bit codes (bytes of x, each < 8) -> 24 bits, code j at bits 3j: pairs, then quads, then
+// the eight, each step moving the upper half down next to the lower one.
+__device__ __forceinline__ uint32_t pack8_3bit(uint2 v) {
+  uint64_t x = static_cast<uint64_t>(v.x) | (static_cast<uint64_t>(v.y) << 32);
+  x = (x | (x >> 5)) & 0x003F003F003F003Full;
+  x = (x | (x >> 10)) & 0x00000FFF00000FFFull;
+  x = (x | (x >> 20)) & 0xFFFFFFull;
+  return static_cast<uint32_t>(x);
+}
+
+// One thread per group of 32 codes of a row (32 bytes) -> three 32-bit words: the group's codes
+// as one 96-bit little-endian number, code i in bits 3i .. 3i + 2.
+__global__ void __launch_bounds__(256)
+pack_codes_3bit_kernel(const uint8_t* __restrict__ codes, int64_t rows, int64_t groups_per_row,
+                       int64_t ldc, uint32_t* __restrict__ packed, int32_t* info) {
+  griddep_wait();
+  const int64_t total = rows * groups_per_row;
+  bool bad = false;
+  for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < total;
+       k += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = k / groups_per_row, gk = k - r * groups_per_row;
+    const uint2* src = reinterpret_cast<const uint2*>(codes + r * ldc + 32 * gk);
+    uint32_t q[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const uint2 v = __ldg(src + i);
+      bad |= ((v.x | v.y) & 0xF8F8F8F8u) != 0u;
+      q[i] = pack8_3bit(make_uint2(v.x & 0x07070707u, v.y & 0x07070707u));
+    }
+    uint32_t* dst = packed + 3 * k;         // rows are dense: 3 words per group
+    dst[0] = q[0] | (q[1] << 24);
+    dst[1] = (q[1] >> 8) | (q[2] << 16);
+    dst[2] = (q[2] >> 16) | (q[3] << 8);
   }
   if (bad) record_info(info, GPTQ_INFO_BAD_CODE);
   griddep_launch_dependents();
@@ -397,6 +439,14 @@ gptq_status run_pack_codes_4bit(const uint8_t* codes, int64_t rows, int64_t cols
   if (blocks > cap) blocks = cap;
   return launch_pdl(pack_codes_4bit_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
                     stream, codes, rows, cols / 8, ldc, packed, info);
+}
+
+gptq_status run_pack_codes_3bit(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ldc,
+                                uint32_t* packed, int32_t* info, cudaStream_t stream) {
+  const int64_t total = rows * (cols / 32);
+  const int64_t blocks = std::min<int64_t>((total + 255) / 256, 16 * num_sms());
+  return launch_pdl(pack_codes_3bit_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0,
+                    stream, codes, rows, cols / 32, ldc, packed, info);
 }
 
 gptq_status run_w4a16_gemv(const uint32_t* packed, const float* scales, const uint8_t* zeros,

@@ -100,6 +100,12 @@ def test_w4a16_entry_points_reject_bad_arguments(built_lib):
     assert pack(FAKE, 4, 64, 60, FAKE, None, None) == _lib.GPTQ_EINVAL      # ldc < cols
     assert pack(FAKE, 4, 64, 68, FAKE, None, None) == _lib.GPTQ_EINVAL      # ldc % 8
     assert pack(FAKE, 0, 64, 64, FAKE, None, None) == _lib.GPTQ_OK          # empty: no-op
+    pack3 = lib.gptq_pack_codes_3bit
+    assert pack3(None, 4, 64, 64, FAKE, None, None) == _lib.GPTQ_EINVAL
+    assert pack3(None, 0, 64, 64, None, None, None) == _lib.GPTQ_OK         # empty, no buffers
+    assert pack3(FAKE, 4, 48, 64, FAKE, None, None) == _lib.GPTQ_EINVAL     # cols % 32
+    assert pack3(FAKE, 4, 64, 60, FAKE, None, None) == _lib.GPTQ_EINVAL     # ldc < cols
+    assert pack3(FAKE, 4, 64, 68, FAKE, None, None) == _lib.GPTQ_EINVAL     # ldc % 8
     mm = lib.gptq_w4a16_matmul
 
     def call(rows=64, cols=256, group=128, dtype=BF, n=1, ldx=256, ldy=64, x=FAKE):
@@ -115,7 +121,7 @@ def test_w4a16_entry_points_reject_bad_arguments(built_lib):
     assert call(ldy=10) == _lib.GPTQ_EINVAL                              # ldy < rows
     assert call(n=-1) == _lib.GPTQ_EINVAL
     assert call(dtype=F32) == _lib.GPTQ_EUNSUPPORTED
-    assert call(n=17) == _lib.GPTQ_EUNSUPPORTED
+    assert call(n=65535 * 128 + 1) == _lib.GPTQ_EUNSUPPORTED          # past the product's grid
     assert call(cols=(1 << 22) + 128, ldx=(1 << 22) + 128) == _lib.GPTQ_EUNSUPPORTED
     assert call(rows=0) == _lib.GPTQ_OK and call(n=0) == _lib.GPTQ_OK    # empty: no-op
     assert call(n=0, x=None) == _lib.GPTQ_OK
