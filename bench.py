@@ -376,6 +376,35 @@ def bench_w4a16(dev, stream, peaks, peaks_src, iters=50):
         out["cases"].append({"layer": name, "n": n, "us": us, "bytes": nbytes,
                              "achieved_gbs": gbs, "frac": gbs / hbm,
                              "weights_per_s": rows * cols / (us * 1e-6)})
+    # batches of activation rows (n > 16): the tensor-core form of the same product; algorithmic
+    # work 2 n rows cols flop (bf16 tensor peak) and the same weight bytes (HBM peak)
+    bf16 = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    key = (12288, 49152, 128, 1)
+    if key not in made:
+        made.clear()
+        torch.cuda.empty_cache()
+        made[key] = [make(12288, 49152, 128, 100)]
+    out["gemm"] = {"kernel": "w4a16_gemm_kernel", "peak_tflops": bf16,
+                   "peak_source": f"{peaks_src} bf16 burst (kernel timed alone)", "cases": []}
+    for n in (64, 256):
+        rows, cols, group = key[:3]
+        _, packed, scales, zeros = made[key][0]
+        X = synth.inputs_torch(synth.scaled_spec(synth.ATTN, 1, cols, n), 7, dev)
+        Y = torch.empty(n, rows, device=dev)
+
+        def fg(k, packed=packed, scales=scales, zeros=zeros, X=X, Y=Y):
+            _lib.w4a16_matmul(packed, scales, zeros, group, X, Y, info, stream)
+
+        us = timed(fg, 20)
+        G = cols // group
+        nbytes = rows * cols / 2 + 5.0 * rows * G + 2.0 * n * cols + 4.0 * n * rows
+        flops = 2.0 * n * rows * cols
+        out["gemm"]["cases"].append({
+            "layer": "fc2_12288x49152_g128", "n": n, "us": us, "bytes": nbytes,
+            "achieved_gbs": nbytes / (us * 1e-6) / 1e9, "frac_hbm": nbytes / (us * 1e-6) / 1e9 / hbm,
+            "achieved_tflops": flops / (us * 1e-6) / 1e12,
+            "frac_tensor": flops / (us * 1e-6) / 1e12 / bf16,
+            "weights_per_s": rows * cols / (us * 1e-6)})
     # packing the quantizer's uint8 codes: reads rows * cols bytes, writes half of that
     made.clear()
     codes, packed, _, _ = make(12288, 49152, 128, 99)
@@ -388,6 +417,19 @@ def bench_w4a16(dev, stream, peaks, peaks_src, iters=50):
     out["pack"] = {"kernel": "pack_codes_4bit_kernel", "layer": "12288x49152", "us": us,
                    "bytes": nbytes, "achieved_gbs": nbytes / (us * 1e-6) / 1e9,
                    "frac": nbytes / (us * 1e-6) / 1e9 / hbm}
+    # the 3-bit layout of the same layer's codes (values < 8): reads one byte per code, writes 3/8
+    codes.bitwise_and_(7)
+    packed3 = torch.empty(codes.shape[0], 3 * codes.shape[1] // 32, device=dev, dtype=torch.int32)
+
+    def fp3(k):
+        _lib.pack_codes_3bit(codes, packed3, info, stream)
+
+    us = timed(fp3, 20)
+    nbytes = 1.375 * codes.numel()
+    out["pack3"] = {"kernel": "pack_codes_3bit_kernel", "layer": "12288x49152", "us": us,
+                    "bytes": nbytes, "achieved_gbs": nbytes / (us * 1e-6) / 1e9,
+                    "frac": nbytes / (us * 1e-6) / 1e9 / hbm}
+    del packed3
     torch.cuda.synchronize(dev)
     if int(info.item()) != 0:
         raise RuntimeError(f"device status {int(info.item())} in the W4A16 leg")
@@ -1004,8 +1046,9 @@ def run_ours(args):
         torch.cuda.synchronize(dev)
         e_ms, _ = aggregate(a.elapsed_time(b), 0, world, dev)
         h2d = Xh.numel() * Xh.element_size() + Wh.numel() * Wh.element_size()
+        # the host receives codes, scales, zeros and err_sq (W_hat = s (q - z) stays on the device)
         d2h = sum(t.numel() * t.element_size() for t in (out.codes, out.scales, out.zeros,
-                                                         out.W_hat, out.err_sq))
+                                                         out.err_sq))
         line["e2e"] = {"value": world * rows * cols * k_e2e / (e_ms / 1e3), "unit": UNIT,
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "steps": k_e2e, "ms_per_step": e_ms / k_e2e}

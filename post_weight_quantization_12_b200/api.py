@@ -6,14 +6,15 @@
     out = q.quantize(W, bits=4, group=128, block=128)   # W [rows, cols] host or device
 
 Host tensors are copied to the device (pinned-memory, non-blocking) before the call; outputs stay
-on the device unless `to_host=True`. PyTorch only provides memory and streams here; every step of
-the method runs in the library's kernels.
+on the device unless `to_host=True` (W_hat, which s (q - z) of the returned codes gives, only with
+`host_w_hat=True`). PyTorch only provides memory and streams here; every step of the method runs in
+the library's kernels.
 
 A 4-bit result can be packed for the W4A16 product, and weights and calibration inputs can be
 rotated before quantization:
 
     lin = pack_4bit(out)                      # PackedLinear4: packed codes, scales, zeros
-    Y = lin(X)                                # fp32 [n, rows] = X W_hat^T for bf16 X [n <= 16, cols]
+    Y = lin(X)                                # fp32 [n, rows] = X W_hat^T for bf16 X [n, cols]
     Wr, Xr = rotate(W, signs), rotate(X, signs)   # data-free randomized Hadamard rotation
 """
 from __future__ import annotations
@@ -118,7 +119,11 @@ class LayerQuantizer:
         return self.S
 
     def quantize(self, W: torch.Tensor, bits: int = 4, group: int = 128, block: int = 128,
-                 to_host: bool = False) -> QuantizedLayer:
+                 to_host: bool = False, host_w_hat: bool = False) -> QuantizedLayer:
+        """Quantize W [rows, cols] against the prepared factor. Outputs stay on the device unless
+        `to_host`; then codes, scales, zeros and err_sq come back in pinned host memory, and W_hat
+        (fp32, the largest output, equal to s (q - z) of the returned codes) only with
+        `host_w_hat` -- otherwise it stays on the device."""
         if self.R is None:
             self.prepare()
         W = self._on_device(W)
@@ -139,7 +144,10 @@ class LayerQuantizer:
             stream = self.stream if self.stream is not None else torch.cuda.current_stream(dev)
             outs = []
             with torch.cuda.stream(stream):
-                for t in (codes, scales, zeros, W_hat, err_sq):
+                for t in (codes, scales, zeros, W_hat if host_w_hat else None, err_sq):
+                    if t is None:
+                        outs.append(W_hat)
+                        continue
                     h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
                     h.copy_(t, non_blocking=True)
                     outs.append(h)
@@ -170,7 +178,8 @@ class PackedLinear4:
         return 8 * self.packed.shape[1]
 
     def __call__(self, X: torch.Tensor, out=None, stream=None) -> torch.Tensor:
-        """fp32 [n, rows] = X W_hat^T for bf16 activations X [n, cols], n <= 16."""
+        """fp32 [n, rows] = X W_hat^T for bf16 activations X [n, cols] (n > 16 on the tensor-core
+        kernel)."""
         if out is None:
             out = torch.empty(X.shape[0], self.rows, device=X.device, dtype=torch.float32)
         _lib.w4a16_matmul(self.packed, self.scales, self.zeros, self.group, X, out, stream=stream)

@@ -24,7 +24,11 @@ def test_host_chunks_match_device_inputs():
     S1 = torch.tril(chunked.S).double().cpu().numpy()
     S2 = torch.tril(whole.S).double().cpu().numpy()
     assert np.linalg.norm(S1 - S2) <= 1e-5 * np.linalg.norm(S2)
-    out_h = chunked.quantize(W, bits=4, group=128, block=128, to_host=True)
+    out_h = chunked.quantize(W, bits=4, group=128, block=128, to_host=True, host_w_hat=True)
+    # without host_w_hat the largest output stays on the device (the host gets what defines it)
+    out_k = chunked.quantize(W, bits=4, group=128, block=128, to_host=True)
+    assert out_k.codes.device.type == "cpu" and out_k.W_hat.device.type == "cuda"
+    assert np.array_equal(out_k.codes.numpy(), out_h.codes.numpy())
     out_d = whole.quantize(W.to(DEV), bits=4, group=128, block=128)
     assert out_h.info == 0 and out_d.info == 0
     assert out_h.codes.device.type == "cpu" and out_h.W_hat.device.type == "cpu"
