@@ -388,6 +388,18 @@ uint64_t gptq_kernel_launches(void);
 gptq_status gptq_selftest_wait_timeout(int32_t* info_dev, int limit_ms, void* stream);
 
 /*
+ * Self-test of the bounded waits on flags in global memory, the form the fused factorization
+ * step uses between its CTAs (no counterpart on the pages). Enqueues one thread that waits for
+ * *flag_dev >= 1 (flag_dev: a caller-owned, 4-byte aligned device int32), reading it with acquire
+ * semantics; if it has not reached 1 after limit_ms milliseconds (1..10000) the thread writes
+ * GPTQ_INFO_TIMEOUT into *info_dev and returns, leaving the context usable. With *flag_dev >= 1
+ * it returns at once and leaves *info_dev alone. Errors: GPTQ_EINVAL for null or misaligned
+ * pointers or a limit out of range, GPTQ_ECUDA for a launch failure.
+ */
+gptq_status gptq_selftest_flag_timeout(const int32_t* flag_dev, int32_t* info_dev, int limit_ms,
+                                       void* stream);
+
+/*
  * Self-test of the tensor-core matrix product every S3-S5 and S8 step runs on (no counterpart on
  * the pages). Computes, in the 3xTF32 scheme (operands split into tf32 big/small parts; the
  * small*small term is dropped):

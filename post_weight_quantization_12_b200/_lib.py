@@ -49,6 +49,7 @@ SIGNATURES = {
     "gptq_selftest_gemm": (_I32, [_P, _I64, _I32, _P, _I64, _I32, _P, _I64, _I32, _I32, _I32,
                                   _F, _F, _I32, _I32, _I32, _P, _P, _P, _SZ, _P, _P]),
     "gptq_selftest_wait_timeout": (_I32, [_P, _I32, _P]),
+    "gptq_selftest_flag_timeout": (_I32, [_P, _P, _I32, _P]),
 }
 
 _lib = None
@@ -96,6 +97,12 @@ def selftest_wait_timeout(info, limit_ms: int, stream=None):
     """Enqueue a bounded wait that nothing will satisfy; it must end with GPTQ_INFO_TIMEOUT."""
     _check(load().gptq_selftest_wait_timeout(_ptr(info), int(limit_ms), _stream(stream)),
            "gptq_selftest_wait_timeout")
+
+
+def selftest_flag_timeout(flag, info, limit_ms: int, stream=None):
+    """One device thread waits (bounded) for the int32 flag to reach 1 (gptq_selftest_flag_timeout)."""
+    _check(load().gptq_selftest_flag_timeout(_ptr(flag), _ptr(info), int(limit_ms), _stream(stream)),
+           "gptq_selftest_flag_timeout")
 
 
 def _check(st: int, where: str):

@@ -29,6 +29,16 @@ __global__ void selftest_wait_kernel(int32_t* info, uint64_t limit_ns) {
   __syncthreads();
 }
 
+// One thread waits for a flag in global memory to reach 1; unless something sets it, the bounded
+// wait must give up and report.
+__global__ void selftest_flag_kernel(const int32_t* flag, int32_t* info, uint64_t limit_ns) {
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    flag_wait_bounded(flag, 1, &abort_flag, info, limit_ns);
+  }
+}
+
 gptq_status set_max_dynamic_smem(const void* kernel, int bytes) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GPTQ_ECUDA;
@@ -296,6 +306,17 @@ gptq_status gptq_selftest_wait_timeout(int32_t* info_dev, int limit_ms, void* st
   if (info_dev == nullptr || limit_ms < 1 || limit_ms > 10000) return GPTQ_EINVAL;
   selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
       info_dev, static_cast<uint64_t>(limit_ms) * 1000000ull);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
+}
+
+gptq_status gptq_selftest_flag_timeout(const int32_t* flag_dev, int32_t* info_dev, int limit_ms,
+                                       void* stream) {
+  if (flag_dev == nullptr || info_dev == nullptr || limit_ms < 1 || limit_ms > 10000)
+    return GPTQ_EINVAL;
+  if (!aligned(flag_dev, 4)) return GPTQ_EINVAL;
+  selftest_flag_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      flag_dev, info_dev, static_cast<uint64_t>(limit_ms) * 1000000ull);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? GPTQ_OK : GPTQ_ECUDA;
 }

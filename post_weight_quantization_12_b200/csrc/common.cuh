@@ -30,6 +30,15 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The dynamic shared memory rounded up to kAlign bytes, formed as an offset from the array itself
+// (not through an integer round trip) so the compiler still knows every access through it is a
+// shared-memory access.
+template <uint32_t kAlign>
+__device__ __forceinline__ uint8_t* smem_align(uint8_t* smem_raw) {
+  const uint32_t mis = smem_u32(smem_raw) & (kAlign - 1u);
+  return smem_raw + ((kAlign - mis) & (kAlign - 1u));
+}
+
 // ------------------------------------------------------------------------------------------------
 // mbarrier
 // ------------------------------------------------------------------------------------------------
@@ -89,6 +98,43 @@ __device__ __forceinline__ bool mbar_drain_bounded(uint64_t* bar, uint32_t parit
     if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
   }
   return true;
+}
+
+// ------------------------------------------------------------------------------------------------
+// Flags in global memory between the CTAs of one launch
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_release_gpu(int32_t* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// order this thread's generic-proxy global accesses with its async-proxy (TMA) ones
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// Wait until *flag >= target (a flag another CTA of the same launch stores with release
+// semantics); bounded like the mbarrier waits.
+__device__ __forceinline__ bool flag_wait_bounded(const int32_t* flag, int target,
+                                                  volatile int* abort_flag, int32_t* info,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+  if (ld_acquire_gpu(flag) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t n = 1;; ++n) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(flag) >= target) return true;
+    if ((n & 15u) == 0) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort_flag = 1;
+        record_info(info, GPTQ_INFO_TIMEOUT);
+        return false;
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------------------------------------------

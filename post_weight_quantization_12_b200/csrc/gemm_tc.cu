@@ -93,8 +93,7 @@ gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ 
   const int n_chunks = (nk + kChunkStages - 1) / kChunkStages;
 
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = smem_align<1024>(smem_raw);
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
   __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
   __shared__ uint32_t tmem_base_sh;
@@ -321,8 +320,7 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
                      const __grid_constant__ CUtensorMap tC, TcGemmParams p, int32_t* info) {
   using namespace tgp;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = smem_align<1024>(smem_raw);
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
   __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
   __shared__ __align__(8) uint64_t cbox[4];        // box j may be written (and holds C if beta != 0)

@@ -84,8 +84,7 @@ hessian_syrk_bf16_tc(const __grid_constant__ CUtensorMap tmap, float* __restrict
                      int n_kblocks, int n_super, int n_s, int32_t* info) {
   using namespace syrk;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = smem_align<1024>(smem_raw);
 
   __shared__ __align__(8) uint64_t full_bar[kStages];    // used in the first CTA
   __shared__ __align__(8) uint64_t empty_bar[kStages];   // in both CTAs

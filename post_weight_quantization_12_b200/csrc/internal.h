@@ -64,6 +64,17 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream);
 gptq_status launch_split_tf32(const float* X, int64_t ldx, int64_t rows, int64_t cols, float* big,
                               float* small, int64_t ldo, cudaStream_t stream);
 
+// S3/S5: steps 0 .. T-2 of the blocked Cholesky of A (n x n, n % 4 == 0, T = ceil(n / 128) >= 2)
+// as fused launches (potrf_step.cu). On entry X_00's split is at (Vb, Vs) (block 0 of an n x n
+// matrix with ld ld_dinv when per_block, else parity 0 of two stacked 128 x 128 blocks), the
+// first panel's split at parity 0 of (Pb, Ps) (two stacked n x 128 buffers, absolute rows) and
+// flags[0 .. T) is zero. Fills L's split (Lb, Ls; n x n), the inverses of the diagonal blocks,
+// and, with store_l, L in A.
+gptq_status launch_potrf_fused(float* A, int64_t n, float* Lb, float* Ls, float* Vb, float* Vs,
+                               int64_t ld_dinv, bool per_block, float* Pb, float* Ps,
+                               int32_t* flags, int32_t* info, int info_base, int rev_n,
+                               bool store_l, cudaStream_t stream);
+
 // S2-S5
 size_t prepare_workspace_bytes(int64_t cols);
 gptq_status run_prepare_hinv(float* S_H, float* R, int64_t cols, int64_t n_total, float damp_rel,

@@ -68,8 +68,7 @@ w4a16_gemm_kernel(const __grid_constant__ CUtensorMap tcodes, const __grid_const
   using C = Cfg<N>;
   constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* smem = smem_align<1024>(smem_raw);
   // A tiles b = 0, 1 (32 KB each), then ring stage s: X (N x 256 B) | codes (8 KB); every part
   // 1024-byte aligned
   auto a_tile = [&](int b) { return smem + b * kABytes; };

@@ -88,6 +88,11 @@ def test_other_entry_points_reject_bad_arguments(built_lib):
                                  FAKE, FAKE, None, FAKE, 16, FAKE, None)
     assert st == _lib.GPTQ_EWORKSPACE
     assert lib.gptq_selftest_wait_timeout(FAKE, 0, None) == _lib.GPTQ_EINVAL
+    assert lib.gptq_selftest_flag_timeout(None, FAKE, 50, None) == _lib.GPTQ_EINVAL
+    assert lib.gptq_selftest_flag_timeout(FAKE, None, 50, None) == _lib.GPTQ_EINVAL
+    assert lib.gptq_selftest_flag_timeout(FAKE, FAKE, 0, None) == _lib.GPTQ_EINVAL
+    assert lib.gptq_selftest_flag_timeout(ctypes.c_void_p(0x10002), FAKE, 50, None) == \
+        _lib.GPTQ_EINVAL
 
 
 def test_w4a16_entry_points_reject_bad_arguments(built_lib):

@@ -245,6 +245,22 @@ def test_bounded_wait_reports_timeout():
     assert float((x * 2).sum().item()) == 8.0
 
 
+def test_flag_wait_reports_timeout():
+    """The bounded wait on a global-memory flag (the fused factorization step's panel flags)."""
+    flag = torch.zeros(1, dtype=torch.int32, device=DEV)
+    info = new_info()
+    _lib.selftest_flag_timeout(flag, info, 50)
+    torch.cuda.synchronize()
+    assert info.item() == _lib.GPTQ_INFO_TIMEOUT
+    flag.fill_(1)
+    info = new_info()
+    _lib.selftest_flag_timeout(flag, info, 50)
+    torch.cuda.synchronize()
+    assert info.item() == 0
+    x = torch.ones(4, device=DEV)
+    assert float((x * 2).sum().item()) == 8.0
+
+
 def test_deterministic_repeat():
     spec = synth.scaled_spec(synth.ATTN, 128, 512, 4096)
     X = synth.inputs_np(spec, 9)
