@@ -216,61 +216,30 @@ struct Split {
   float* s;
 };
 
-// Blocked right-looking Cholesky of A (n x n, lower, in place).
-//   Lsp:  tf32 split of L's panels (n x n, ld n), written as the panels are solved;
-//   Dsp:  where each diagonal block's inverse goes (ld ld_dinv): at block k0 of an n x n matrix
-//         when per_block is set (the block diagonal of L^-1), else one shared 128 x 128 scratch;
-//   Psp:  split of the current panel before its solve (n x 128);
+// Blocked right-looking Cholesky of A (n x n, lower, in place; n % 4 == 0, A 16-byte aligned),
+// 128-wide blocks: the diagonal block 0 and the split of the first panel, then one fused launch
+// per step (potrf_step.cu).
+//   Lsp:   tf32 split of L's panels (n x n, ld n), written as the panels are solved;
+//   Dsp:   where each diagonal block's inverse goes (ld ld_dinv): at block k0 of an n x n matrix
+//          when per_block is set (the block diagonal of L^-1), else two 128 x 128 scratch blocks
+//          used in turn;
+//   Psp:   the split of the next panel, two n x 128 buffers used in turn (absolute rows);
+//   flags: ceil(n / 128) ints, the steps' panel flags;
 //   rev_n: > 0 when A is the order-reversed matrix (pivot codes then name original columns);
-//   store_l: write the factored diagonal blocks back into A (only needed when A's own lower
-//         triangle is the result; the panels below them are always written).
+//   store_l: write L back into A (only needed when A's own lower triangle is the result).
 static gptq_status potrf_blocked(float* A, int64_t n, Split Lsp, Split Dsp, int64_t ld_dinv,
-                                 bool per_block, Split Psp, int32_t* info, int info_base,
-                                 int rev_n, bool store_l, cudaStream_t stream) {
-  using namespace la;
-  for (int64_t k0 = 0; k0 < n; k0 += kNB) {
-    const int nb = static_cast<int>(n - k0 < kNB ? n - k0 : kNB);
-    const int64_t doff = per_block ? k0 * ld_dinv + k0 : 0;
-    GPTQ_TRY(launch_potrf_diag(A, n, static_cast<int>(k0), nb, Dsp.b + doff, Dsp.s + doff, ld_dinv,
-                               info, info_base, rev_n, store_l, stream));
-    const int64_t m = n - k0 - nb;
-    if (m == 0) break;
-    float* A21 = A + (k0 + nb) * n + k0;
-    GPTQ_TRY(launch_split_tf32(A21, n, m, nb, Psp.b, Psp.s, kNB, stream));
-    // panel solve: L21 = A21 * Dinv^T, written to A and, split, to Lsp
-    const int64_t loff = (k0 + nb) * n + k0;
-    TcGemmArgs t{Psp.b, Psp.s, Dsp.b + doff, Dsp.s + doff, kNB, ld_dinv, 0, 0,
-                 static_cast<int>(m), nb, nb, 1.f, 0.f, 0, 0, 0,
-                 A21, n, Lsp.b + loff, Lsp.s + loff, n, info};
-    GPTQ_TRY(launch_gemm_tc(t, stream));
-    // trailing update: A22 -= L21 L21^T (lower tiles)
-    TcGemmArgs u{Lsp.b + loff, Lsp.s + loff, Lsp.b + loff, Lsp.s + loff, n, n, 0, 0,
-                 static_cast<int>(m), static_cast<int>(m), nb, -1.f, 1.f, 1, 0, 0,
-                 A + (k0 + nb) * n + (k0 + nb), n, nullptr, nullptr, 0, info};
-    GPTQ_TRY(launch_gemm_tc(u, stream));
-  }
-  return GPTQ_OK;
-}
-
-// The same factorization with steps 0 .. T-2 fused (see potrf_step.cu): the diagonal block 0 and
-// the split of the first panel, then one launch per step. Needs n % 4 == 0 (TMA row pitch),
-// n > 128 and 16-byte aligned buffers; Psp holds two n x 128 parities, Dsp (when not per block)
-// two 128 x 128 ones, flags ceil(n / 128) ints.
-static gptq_status potrf_fused(float* A, int64_t n, Split Lsp, Split Dsp, int64_t ld_dinv,
-                               bool per_block, Split Psp, int32_t* flags, int32_t* info,
-                               int info_base, int rev_n, bool store_l, cudaStream_t stream) {
+                                 bool per_block, Split Psp, int32_t* flags, int32_t* info,
+                                 int info_base, int rev_n, bool store_l, cudaStream_t stream) {
   using namespace la;
   const int T = static_cast<int>((n + kNB - 1) / kNB);
-  GPTQ_TRY(launch_potrf_diag(A, n, 0, kNB, Dsp.b, Dsp.s, ld_dinv, info, info_base, rev_n, store_l,
+  const int nb0 = static_cast<int>(n < kNB ? n : kNB);
+  GPTQ_TRY(launch_potrf_diag(A, n, 0, nb0, Dsp.b, Dsp.s, ld_dinv, info, info_base, rev_n, store_l,
                              stream, flags, T));
+  if (T == 1) return GPTQ_OK;
   GPTQ_TRY(launch_split_tf32(A + kNB * n, n, n - kNB, kNB, Psp.b + kNB * kNB, Psp.s + kNB * kNB,
                              kNB, stream));
   return launch_potrf_fused(A, n, Lsp.b, Lsp.s, Dsp.b, Dsp.s, ld_dinv, per_block, Psp.b, Psp.s,
                             flags, info, info_base, rev_n, store_l, stream);
-}
-
-static bool fused_ok(const float* A, int64_t n) {
-  return n % 4 == 0 && n > la::kNB && (reinterpret_cast<uintptr_t>(A) & 15) == 0;
 }
 
 namespace {
@@ -368,12 +337,8 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
 
   // S3: H_d = L L^T in R (reversed route: J H_d J = M M^T, M written as L below); the inverses of
   // L's diagonal blocks land in V (the split of L^-1)
-  if (fused_ok(R, n))
-    GPTQ_TRY(potrf_fused(R, n, w.L, w.V, n, true, w.P, w.flags, info, 0,
+  GPTQ_TRY(potrf_blocked(R, n, w.L, w.V, n, true, w.P, w.flags, info, 0,
                          reversed ? static_cast<int>(n) : 0, false, stream));
-  else
-    GPTQ_TRY(potrf_blocked(R, n, w.L, w.V, n, true, w.P, info, 0,
-                           reversed ? static_cast<int>(n) : 0, false, stream));
 
   // S4a: the rest of L^-1 by recursive doubling over the diagonal blocks already inverted.
   GPTQ_TRY(trtri_doubling(w, n, info, stream));
@@ -391,12 +356,8 @@ gptq_status run_prepare_hinv(float* S_H, float* R, int64_t n, int64_t n_total, f
   GPTQ_TRY(launch_gemm_tc(h, stream));
 
   // S5: H_d^-1 = L2 L2^T (reusing the L split and the diagonal scratch), then R = L2^T
-  if (fused_ok(R, n))
-    GPTQ_TRY(potrf_fused(R, n, w.L, w.D, kNB, false, w.P, w.flags, info, static_cast<int>(n), 0,
+  GPTQ_TRY(potrf_blocked(R, n, w.L, w.D, kNB, false, w.P, w.flags, info, static_cast<int>(n), 0,
                          true, stream));
-  else
-    GPTQ_TRY(potrf_blocked(R, n, w.L, w.D, kNB, false, w.P, info, static_cast<int>(n), 0, true,
-                           stream));
   return launch_pdl(transpose_to_upper_kernel, dim3(ntri), dim3(32, 8), 0, stream, R, n);
 }
 
