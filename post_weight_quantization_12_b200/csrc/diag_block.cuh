@@ -38,8 +38,8 @@ __device__ __forceinline__ void decode_tri(int t, int& I, int& J) {
 // S3/S5 diagonal block: Cholesky of A[k0:k0+nb, k0:k0+nb] on chip (lower; the block's strict upper
 // part is zeroed in A when store_l is set) and the tf32 split of its triangular inverse into
 // (Db, Ds) with ld ldd. Blocked by 32-column pieces; for each piece kb:
-//  F  warps 0-3 factor the piece and build its inverse in the same loop, four columns per step
-//     (factor_piece4_mw).
+//  F  warps 0-3 factor the piece and build its inverse in the same loop, eight columns per step
+//     (factor_piece8_mw).
 //     Meanwhile warps 4-15 finish the previous piece's trailing update beyond this piece's
 //     columns and form the block's inverse row blocks,
 //     X[b][j] = -X[b][b] * sum_m L[b][m] X[m][j]: the sum for row block kb and the product with
@@ -111,32 +111,32 @@ __device__ __forceinline__ void inverse_row_product(float* X, const float* OT, i
     for (int v = 0; v < 4; ++v) X[(r0 + u) * LD + 4 * jg + v] = -acc[u][v];
 }
 
-// Factor and invert one 32 x 32 piece, four columns per step, on warps 0-3. Lane l is row l; each
+// Factor and invert one 32 x 32 piece, eight columns per step, on warps 0-3. Lane l is row l; each
 // register holds L[l][k] for k < l (the factor's row) or the running sum for X[k][l] for k > l (the
 // inverse's column, X[j][t] = (delta_jt - sum_{m<j} L[j][m] X[m][t]) / L[j][j]); the diagonal
-// pair L[l][l], X[l][l] ends in ldiag / xdiag. Per step the owning warp factors the step's 4 x 4
-// diagonal block itself (broadcast by shuffles) and solves every row's four entries of L or X;
-// entries of L then take -L[l][j] L[k][j] and entries of X take L[k][j] X[j][l], so one FMA per
-// register and column serves both. A pivot that is not positive is replaced by 1 and its index
-// goes to badj. Warp w keeps columns 8w .. 8w+7 of every row in e[0..7]; step t (columns
-// 4t .. 4t+3) belongs to warp t/2, which publishes every row's entries of L (A4) and of X (X4) for
-// the step; after a barrier of the four warps each warp applies them to its later columns.
+// pair L[l][l], X[l][l] ends in ldiag / xdiag. Warp w keeps columns 8w .. 8w+7 of every row in
+// e[0..7] and owns step w: it factors the step's 8 x 8 diagonal block itself (broadcast by
+// shuffles), solves every row's eight entries of L or X and publishes them (A8, X8: two float4
+// per row); after a barrier of the four warps each later warp applies them to its own columns:
+// entries of L take -L[l][j] L[k][j] and entries of X take L[k][j] X[j][l], one FMA per register
+// and column for both. A pivot that is not positive is replaced by 1 and its index goes to badj.
+// (Four columns per step, eight steps, measured 7.4 k cycles for the first piece; this form 6.9 k.)
 // ldiag / xdiag are valid in the warp that owns column `lane`.
-__device__ __forceinline__ void factor_piece4_mw(float (&e)[8], float& ldiag, float& xdiag,
-                                                 int& badj, float4* A4, float4* X4, int warp,
+__device__ __forceinline__ void factor_piece8_mw(float (&e)[8], float& ldiag, float& xdiag,
+                                                 int& badj, float4* A8, float4* X8, int warp,
                                                  int lane) {
 #pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    const int j = 4 * t, q0 = (t & 1) * 4;
-    if (warp == (t >> 1)) {
-      float b[4][4];
+  for (int t = 0; t < 4; ++t) {
+    const int j = 8 * t;
+    if (warp == t) {
+      float b[8][8];
 #pragma unroll
-      for (int p = 0; p < 4; ++p)
+      for (int p = 0; p < 8; ++p)
 #pragma unroll
-        for (int q = 0; q <= p; ++q) b[p][q] = __shfl_sync(0xffffffffu, e[q0 + q], j + p);
-      float lb[4][4], r[4];
+        for (int q = 0; q <= p; ++q) b[p][q] = __shfl_sync(0xffffffffu, e[q], j + p);
+      float lb[8][8], r[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 8; ++q) {
         float d = b[q][q];
 #pragma unroll
         for (int s = 0; s < q; ++s) d = fmaf(-lb[q][s], lb[q][s], d);
@@ -145,18 +145,18 @@ __device__ __forceinline__ void factor_piece4_mw(float (&e)[8], float& ldiag, fl
         lb[q][q] = ok ? d * r[q] : 1.f;
         badj = (!ok && badj == 32) ? j + q : badj;
 #pragma unroll
-        for (int p = q + 1; p < 4; ++p) {
+        for (int p = q + 1; p < 8; ++p) {
           float v = b[p][q];
 #pragma unroll
           for (int s = 0; s < q; ++s) v = fmaf(-lb[p][s], lb[q][s], v);
           lb[p][q] = v * r[q];
         }
       }
-      float a[4], x[4];                    // L[lane][j+q] and X[j+q][lane]
+      float a[8], x[8];                    // L[lane][j+q] and X[j+q][lane]
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < 8; ++q) {
         const int k = j + q;
-        float sa = e[q0 + q], sx = -e[q0 + q];
+        float sa = e[q], sx = -e[q];
 #pragma unroll
         for (int s = 0; s < q; ++s) {
           sa = fmaf(-a[s], lb[q][s], sa);
@@ -165,7 +165,7 @@ __device__ __forceinline__ void factor_piece4_mw(float (&e)[8], float& ldiag, fl
         if (lane > k) {
           a[q] = sa * r[q];
           x[q] = 0.f;
-          e[q0 + q] = a[q];
+          e[q] = a[q];
         } else if (lane == k) {
           a[q] = lb[q][q];
           x[q] = r[q];
@@ -174,26 +174,28 @@ __device__ __forceinline__ void factor_piece4_mw(float (&e)[8], float& ldiag, fl
         } else {
           a[q] = 0.f;
           x[q] = sx * r[q];
-          e[q0 + q] = x[q];
+          e[q] = x[q];
         }
       }
-      A4[t * 32 + lane] = make_float4(a[0], a[1], a[2], a[3]);
-      X4[t * 32 + lane] = make_float4(x[0], x[1], x[2], x[3]);
+      A8[(t * 32 + lane) * 2] = make_float4(a[0], a[1], a[2], a[3]);
+      A8[(t * 32 + lane) * 2 + 1] = make_float4(a[4], a[5], a[6], a[7]);
+      X8[(t * 32 + lane) * 2] = make_float4(x[0], x[1], x[2], x[3]);
+      X8[(t * 32 + lane) * 2 + 1] = make_float4(x[4], x[5], x[6], x[7]);
     }
     named_barrier_or(la::kFactorBar, 128, false);
-    if (warp >= (t >> 1)) {
-      const float4 a4 = A4[t * 32 + lane], x4 = X4[t * 32 + lane];
+    if (warp > t) {
+      const float4 a0 = A8[(t * 32 + lane) * 2], a1 = A8[(t * 32 + lane) * 2 + 1];
+      const float4 x0 = X8[(t * 32 + lane) * 2], x1 = X8[(t * 32 + lane) * 2 + 1];
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
         const int k = 8 * warp + q;
-        if (k > j + 3) {
-          const float4 c = A4[t * 32 + k];
-          const bool fac = lane >= k;
-          e[q] = fmaf(c.x, fac ? -a4.x : x4.x, e[q]);
-          e[q] = fmaf(c.y, fac ? -a4.y : x4.y, e[q]);
-          e[q] = fmaf(c.z, fac ? -a4.z : x4.z, e[q]);
-          e[q] = fmaf(c.w, fac ? -a4.w : x4.w, e[q]);
-        }
+        const float4 c0 = A8[(t * 32 + k) * 2], c1 = A8[(t * 32 + k) * 2 + 1];
+        const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const bool fac = lane >= k;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) e[q] = fmaf(cv[u], fac ? -av[u] : xv[u], e[q]);
       }
     }
   }
@@ -288,7 +290,7 @@ __device__ __forceinline__ void diag_factor_block(float* sm, float4* stepA, floa
       }
       float ldiag = 1.f, xdiag = 1.f;
       int badj = 32;
-      factor_piece4_mw(e, ldiag, xdiag, badj, stepA, stepX, warp, lane);
+      factor_piece8_mw(e, ldiag, xdiag, badj, stepA, stepX, warp, lane);
       if (lane == 0 && badj < 32) atomicMin(&bad, c0 + badj);
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
