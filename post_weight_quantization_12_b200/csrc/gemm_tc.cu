@@ -80,7 +80,11 @@ gemm_tf32x3_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ 
                TcGemmParams p, int32_t* info) {
   using namespace tg;
   const int per_batch = p.tiles_m * p.tiles_n;
-  const int bt = blockIdx.x / per_batch, tix = blockIdx.x - bt * per_batch;
+  const int bt = blockIdx.x / per_batch;
+  // With k stopping after the tile's rows the later row tiles are the longer ones: they take the
+  // first CTAs, so the last wave is made of the short tiles (longest first).
+  const int tix0 = blockIdx.x - bt * per_batch;
+  const int tix = p.khi_from_m ? per_batch - 1 - tix0 : tix0;
   const int tm = tix / p.tiles_n, tn = tix - (tix / p.tiles_n) * p.tiles_n;
   const int m0 = tm * BM, n0 = tn * BN;
   const int boff = bt * p.bstride;          // this batch's shift along the diagonal
