@@ -679,6 +679,266 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
   }
 }
 
+// ------------------------------------------------------------------------------------------------
+// The lazy trailing update's shape (S8: C += alpha * A B with A K-major, B MN-major, K <= 128,
+// whole 128-column tiles, C read and written): the same product with the A row band kept in
+// shared memory. A CTA's tiles are consecutive in row-major order, so most of them share their A
+// band; the band (up to 4 k-blocks x big/small = 128 KB) is loaded once per band and only B is
+// streamed (two 32 KB stages), which halves the operand bytes per tile. C goes through two
+// 128 x 32 boxes that take a tile's four column boxes in turn.
+// ------------------------------------------------------------------------------------------------
+namespace tga {
+constexpr int BM = 128, BN = 128, BK = 32, kMaxKb = 4;
+constexpr int kPartBytes = BM * BK * 4;                 // 16 KB: one part (big or small)
+constexpr int kABytes = kMaxKb * 2 * kPartBytes;        // the A band: k-block kb at kb * 32 KB
+constexpr int kStages = 2;
+constexpr int kStageBytes = 2 * kPartBytes;             // B_big, B_small
+constexpr int kBoxBytes = BM * 32 * 4;                  // 16 KB
+constexpr int kBoxes = 2;
+constexpr int kSmemBytes = kABytes + kStages * kStageBytes + kBoxes * kBoxBytes + 1024;
+constexpr int kThreads = 224;                           // 0 loads, 1 MMA, 2-5 epilogue, 6 C
+constexpr int kIssuerWarp = 6;
+constexpr uint32_t kTmemCols = 512;
+}  // namespace tga
+
+__global__ void __launch_bounds__(tga::kThreads, 1)
+gemm_tf32x3_aband_tc(const __grid_constant__ CUtensorMap tAb, const __grid_constant__ CUtensorMap tAs,
+                     const __grid_constant__ CUtensorMap tBb, const __grid_constant__ CUtensorMap tBs,
+                     const __grid_constant__ CUtensorMap tC, TcGemmParams p, int32_t* info) {
+  using namespace tga;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_align<1024>(smem_raw);
+  uint8_t* sa = smem;                                   // the A band
+  uint8_t* sb = smem + kABytes;                         // B stages
+  uint8_t* cs = sb + kStages * kStageBytes;             // C boxes
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t a_full, a_empty;
+  __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
+  __shared__ __align__(8) uint64_t cbox[kBoxes];        // box b holds the C of its next box
+  __shared__ __align__(8) uint64_t ready[kBoxes];       // box b written by the epilogue
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nk = (p.K + BK - 1) / BK;   // 1..4
+  const int t_begin = static_cast<int>(static_cast<int64_t>(blockIdx.x) * p.n_tiles / gridDim.x);
+  const int t_end = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * p.n_tiles / gridDim.x);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full_bar[s], 1);
+      mbar_init(&empty_bar[s], 1);
+    }
+    mbar_init(&a_full, 1);
+    mbar_init(&a_empty, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 128);
+    }
+    for (int b = 0; b < kBoxes; ++b) {
+      mbar_init(&cbox[b], 1);
+      mbar_init(&ready[b], 128);
+    }
+    mbar_init(&mma_done, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base_sh;
+  griddep_wait();
+  griddep_launch_dependents();
+
+  if (warp == 0) {
+    // ---------------- loads: the A band when it changes, B per tile ----------------
+    if (lane == 0) {
+      int s = 0, issued = 0, bands = 0, band = -1;
+      uint32_t ph = 0;
+      for (int t = t_begin; t < t_end && !abort_flag; ++t) {
+        const int tm = t / p.tiles_n, tn = t - tm * p.tiles_n;
+        const int m0 = tm * BM, n0 = tn * BN;
+        if (tm != band) {
+          // the MMAs of the previous band are done with it
+          if (bands > 0 &&
+              !mbar_wait_bounded(&a_empty, static_cast<uint32_t>((bands - 1) & 1), &abort_flag, info))
+            goto producer_done;
+          mbar_arrive_expect_tx(&a_full, static_cast<uint32_t>(nk) * 2u * kPartBytes);
+          for (int kb = 0; kb < nk; ++kb) {
+            tma_load_2d(sa + kb * 2 * kPartBytes, &tAb, &a_full, kb * BK, m0);
+            tma_load_2d(sa + kb * 2 * kPartBytes + kPartBytes, &tAs, &a_full, kb * BK, m0);
+          }
+          band = tm;
+          ++bands;
+        }
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&empty_bar[s], ph ^ 1u, &abort_flag, info)) goto producer_done;
+          uint8_t* st = sb + s * kStageBytes;
+          mbar_arrive_expect_tx(&full_bar[s], kStageBytes);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            tma_load_2d(st + q * 4096, &tBb, &full_bar[s], n0 + 32 * q, kb * BK);
+            tma_load_2d(st + kPartBytes + q * 4096, &tBs, &full_bar[s], n0 + 32 * q, kb * BK);
+          }
+          ++issued;
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+      }
+    producer_done:
+      for (int i = (issued > kStages ? issued - kStages : 0); i < issued; ++i)
+        mbar_drain_bounded(&full_bar[i % kStages], static_cast<uint32_t>((i / kStages) & 1));
+      if (bands > 0) mbar_drain_bounded(&a_full, static_cast<uint32_t>((bands - 1) & 1));
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = make_idesc(/*tf32*/ 2, 0, 1, BM, BN);
+      int s = 0, c = 0, bands = 0, band = -1;
+      uint32_t ph = 0;
+      for (int t = t_begin; t < t_end && !abort_flag; ++t, ++c) {
+        const int tm = t / p.tiles_n;
+        const int buf = c & 1;
+        if (!mbar_wait_bounded(&acc_empty[buf], ((c >> 1) & 1) ^ 1u, &abort_flag, info))
+          goto mma_finish;
+        if (tm != band) {
+          if (!mbar_wait_bounded(&a_full, static_cast<uint32_t>(bands & 1), &abort_flag, info))
+            goto mma_finish;
+          band = tm;
+          ++bands;
+        }
+        tc_fence_after();
+        const uint32_t t_main = tmem + buf * 256, t_corr = t_main + 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_bounded(&full_bar[s], ph, &abort_flag, info)) goto mma_finish;
+          tc_fence_after();
+          const uint32_t abase = smem_u32(sa + kb * 2 * kPartBytes);
+          const uint32_t bbase = smem_u32(sb + s * kStageBytes);
+#pragma unroll
+          for (int kk = 0; kk < BK / 8; ++kk) {
+            // A K-major (128-byte swizzle, +32 B per 8 k); B MN-major (128-byte swizzle with
+            // 32-byte atoms: 32-element chunks 4 KB apart, +1024 B per 8 k)
+            const uint64_t ab = smem_desc(abase + kk * 32, 16, 1024, kSwizzle128B);
+            const uint64_t as = smem_desc(abase + kPartBytes + kk * 32, 16, 1024, kSwizzle128B);
+            const uint64_t bb = smem_desc(bbase + kk * 1024, 4096, 512, kSwizzle128B32BAtom);
+            const uint64_t bs =
+                smem_desc(bbase + kPartBytes + kk * 1024, 4096, 512, kSwizzle128B32BAtom);
+            const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+            tc_mma_tf32(t_corr, ab, bs, idesc, accum);
+            tc_mma_tf32(t_corr, as, bb, idesc, 1u);
+            tc_mma_tf32(t_main, ab, bb, idesc, accum);
+          }
+          tc_commit(&empty_bar[s]);
+          if (++s == kStages) { s = 0; ph ^= 1u; }
+        }
+        tc_commit(&acc_full[buf]);
+        // the band is released once the last tile using it is done
+        if (t + 1 == t_end || (t + 1) / p.tiles_n != tm) tc_commit(&a_empty);
+      }
+    mma_finish:
+      tc_commit(&mma_done);
+      mbar_drain_bounded(&mma_done, 0);
+    }
+  } else if (warp == kIssuerWarp) {
+    // ---------------- C boxes: a tile's four column boxes go through two buffers in turn ------
+    if (lane == 0) {
+      uint32_t rdy_ph = 0, last_ph = 0, rel = 0;
+      auto release = [&](int t, int j) {   // load the C of box j of tile t into buffer j & 1
+        const int b = j & 1;
+        if (rel & (1u << b)) last_ph ^= 1u << b;
+        rel |= 1u << b;
+        const int tm = t / p.tiles_n, tn = t - tm * p.tiles_n;
+        mbar_arrive_expect_tx(&cbox[b], kBoxBytes);
+        tma_load_2d(cs + b * kBoxBytes, &tC, &cbox[b], tn * BN + 32 * j, tm * BM);
+      };
+      if (t_begin < t_end) {
+        release(t_begin, 0);
+        release(t_begin, 1);
+      }
+      bool ok = true;
+      for (int t = t_begin; ok && t < t_end; ++t) {
+        const int tm = t / p.tiles_n, tn = t - tm * p.tiles_n;
+        for (int j = 0; j < 4; ++j) {
+          const int b = j & 1;
+          if (!mbar_wait_bounded(&ready[b], (rdy_ph >> b) & 1u, &abort_flag, info)) {
+            ok = false;
+            break;
+          }
+          rdy_ph ^= 1u << b;
+          tma_store_2d(&tC, cs + b * kBoxBytes, tn * BN + 32 * j, tm * BM);
+          tma_store_commit();
+          tma_store_wait_read<0>();           // the buffer has left shared memory
+          if (j < 2) release(t, j + 2);
+          else if (t + 1 < t_end) release(t + 1, j - 2);
+        }
+      }
+      tma_store_wait_all();
+      for (int b = 0; b < kBoxes; ++b)
+        if (rel & (1u << b)) mbar_drain_bounded(&cbox[b], (last_ph >> b) & 1u);
+    }
+  } else if (warp >= 2 && warp < 6) {
+    // ---------------- epilogue: fold TMEM, C = alpha * acc + beta * C in the boxes ----------
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t rsw = static_cast<uint32_t>(r & 7);
+    uint32_t tok_ph = 0;
+    int c = 0;
+    for (int t = t_begin; t < t_end; ++t, ++c) {
+      const int buf = c & 1;
+      const bool ok = mbar_wait_bounded(&acc_full[buf], (c >> 1) & 1, &abort_flag, info);
+      if (named_barrier_or(1, 128, !ok || abort_flag)) break;
+      tc_fence_after();
+      float acc[BN];
+      const uint32_t t_main = tmem + buf * 256 + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t vm[32], vc[32];
+        tmem_ld_32x32b_x32(t_main + cc * 32, vm);
+        tmem_ld_32x32b_x32(t_main + 128 + cc * 32, vc);
+        tmem_wait_ld();
+#pragma unroll
+        for (int u = 0; u < 32; ++u) acc[cc * 32 + u] = __uint_as_float(vm[u]) + __uint_as_float(vc[u]);
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[buf]);
+      bool stop = false;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int b = j & 1;
+        const bool okc = !stop && mbar_wait_bounded(&cbox[b], (tok_ph >> b) & 1u, &abort_flag, info);
+        if (okc) {
+          tok_ph ^= 1u << b;
+          uint8_t* rowp = cs + b * kBoxBytes + r * 128;
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            float4* a = reinterpret_cast<float4*>(rowp + ((static_cast<uint32_t>(u) ^ rsw) << 4));
+            const float* x = acc + j * 32 + 4 * u;
+            const float4 o = *a;
+            *a = make_float4(fmaf(p.beta, o.x, p.alpha * x[0]), fmaf(p.beta, o.y, p.alpha * x[1]),
+                             fmaf(p.beta, o.z, p.alpha * x[2]), fmaf(p.beta, o.w, p.alpha * x[3]));
+          }
+        }
+        // every epilogue thread takes the same branch (a lost wait stops all of them)
+        stop = named_barrier_or(1, 128, !okc || abort_flag);
+        if (!stop) {
+          fence_proxy_async_smem();
+          mbar_arrive(&ready[b]);
+        }
+      }
+      if (stop) break;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
 // x -> (tf32(x), x - tf32(x)) for a rows x cols block (row-major, leading dims in elements).
 __global__ void split_tf32_kernel(const float* __restrict__ X, int64_t ldx, int64_t rows,
                                   int64_t cols, float* __restrict__ big, float* __restrict__ small,
@@ -772,6 +1032,15 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
                              tgp::BM, CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK)
       return st;
     const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
+    if (p.stage_c && !g.a_mn && g.b_mn && !g.lower && g.Cbig == nullptr && g.beta != 0.f &&
+        g.N % tga::BN == 0) {
+      // the lazy trailing update's shape: the A band stays in shared memory
+      if ((st = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_tf32x3_aband_tc),
+                                     tga::kSmemBytes)) != GPTQ_OK)
+        return st;
+      return launch_pdl(gemm_tf32x3_aband_tc, dim3(grid), dim3(tga::kThreads), tga::kSmemBytes,
+                        stream, tAb, tAs, tBb, tBs, tC, p, g.info);
+    }
     const int smem = p.stage_c ? tgp::kSmemBytesStaged : tgp::kSmemBytes;
     return launch_pdl(gemm_tf32x3_panel_tc, dim3(grid), dim3(tgp::kThreads), smem, stream, tAb,
                       tAs, tBb, tBs, tC, p, g.info);

@@ -128,6 +128,10 @@ def test_gemm_lower_update_k128(n, K):
     (512, 640, 128, 0, 1.0),     # 640 columns: five 128-wide tile columns
     (256, 256, 64, 1, 0.0),      # C written only
     (1024, 384, 100, 0, 1.0),    # K not a multiple of the 32-wide stage
+    # the lazy-update shape on more tiles than SMs (a CTA's tiles then cross A-band boundaries)
+    (4096, 3968, 128, 1, 1.0),   # the widest update of a 4096-column layer: 992 tiles
+    (1536, 1664, 128, 1, 1.0),   # 156 tiles: a few CTAs take two, some of them in two bands
+    (1000, 2560, 96, 1, 1.0),    # ragged last band and K of three 32-wide stages
 ])
 def test_gemm_k128_shapes(M, N, K, b_mn, beta):
     """K <= 128 products on multi-tile shapes: both B layouts, beta 0 and 1, ragged K."""
