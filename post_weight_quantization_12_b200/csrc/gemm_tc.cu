@@ -681,11 +681,12 @@ gemm_tf32x3_panel_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
 
 // ------------------------------------------------------------------------------------------------
 // The lazy trailing update's shape (S8: C += alpha * A B with A K-major, B MN-major, K <= 128,
-// whole 128-column tiles, C read and written): the same product with the A row band kept in
-// shared memory. A CTA's tiles are consecutive in row-major order, so most of them share their A
-// band; the band (up to 4 k-blocks x big/small = 128 KB) is loaded once per band and only B is
-// streamed (two 32 KB stages), which halves the operand bytes per tile. C goes through two
-// 128 x 32 boxes that take a tile's four column boxes in turn.
+// whole 128-column tiles, beta = 1): the same product with the A row band kept in shared memory.
+// A CTA's tiles are consecutive in row-major order, so most of them share their A band; the band
+// (up to 4 k-blocks x big/small = 128 KB) is loaded once per band and only B is streamed (two
+// 32 KB stages), which halves the operand bytes per tile. C is never read by the CTA: each
+// 128 x 32 box of alpha * acc goes into one of two shared buffers and a TMA reduce-add adds it
+// into C in L2 (one fp32 add per element, the same rounding as reading C and adding).
 // ------------------------------------------------------------------------------------------------
 namespace tga {
 constexpr int BM = 128, BN = 128, BK = 32, kMaxKb = 4;
@@ -714,7 +715,7 @@ gemm_tf32x3_aband_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
   __shared__ __align__(8) uint64_t a_full, a_empty;
   __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], mma_done;
-  __shared__ __align__(8) uint64_t cbox[kBoxes];        // box b holds the C of its next box
+  __shared__ __align__(8) uint64_t cbox[kBoxes];        // box b may be written
   __shared__ __align__(8) uint64_t ready[kBoxes];       // box b written by the epilogue
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
@@ -842,21 +843,11 @@ gemm_tf32x3_aband_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
       mbar_drain_bounded(&mma_done, 0);
     }
   } else if (warp == kIssuerWarp) {
-    // ---------------- C boxes: a tile's four column boxes go through two buffers in turn ------
+    // ---------------- C boxes: a tile's four column boxes go through two buffers in turn, each
+    // added into C by a TMA reduce-add and handed back once it has been read out ----------
     if (lane == 0) {
-      uint32_t rdy_ph = 0, last_ph = 0, rel = 0;
-      auto release = [&](int t, int j) {   // load the C of box j of tile t into buffer j & 1
-        const int b = j & 1;
-        if (rel & (1u << b)) last_ph ^= 1u << b;
-        rel |= 1u << b;
-        const int tm = t / p.tiles_n, tn = t - tm * p.tiles_n;
-        mbar_arrive_expect_tx(&cbox[b], kBoxBytes);
-        tma_load_2d(cs + b * kBoxBytes, &tC, &cbox[b], tn * BN + 32 * j, tm * BM);
-      };
-      if (t_begin < t_end) {
-        release(t_begin, 0);
-        release(t_begin, 1);
-      }
+      uint32_t rdy_ph = 0;
+      for (int b = 0; b < kBoxes; ++b) mbar_arrive(&cbox[b]);
       bool ok = true;
       for (int t = t_begin; ok && t < t_end; ++t) {
         const int tm = t / p.tiles_n, tn = t - tm * p.tiles_n;
@@ -867,19 +858,16 @@ gemm_tf32x3_aband_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
             break;
           }
           rdy_ph ^= 1u << b;
-          tma_store_2d(&tC, cs + b * kBoxBytes, tn * BN + 32 * j, tm * BM);
+          tma_reduce_add_2d(&tC, cs + b * kBoxBytes, tn * BN + 32 * j, tm * BM);
           tma_store_commit();
           tma_store_wait_read<0>();           // the buffer has left shared memory
-          if (j < 2) release(t, j + 2);
-          else if (t + 1 < t_end) release(t + 1, j - 2);
+          mbar_arrive(&cbox[b]);
         }
       }
       tma_store_wait_all();
-      for (int b = 0; b < kBoxes; ++b)
-        if (rel & (1u << b)) mbar_drain_bounded(&cbox[b], (last_ph >> b) & 1u);
     }
   } else if (warp >= 2 && warp < 6) {
-    // ---------------- epilogue: fold TMEM, C = alpha * acc + beta * C in the boxes ----------
+    // ---------------- epilogue: fold TMEM, alpha * acc into the boxes ----------------
     const int q = warp & 3;
     const int r = q * 32 + lane;
     const uint32_t rsw = static_cast<uint32_t>(r & 7);
@@ -915,9 +903,7 @@ gemm_tf32x3_aband_tc(const __grid_constant__ CUtensorMap tAb, const __grid_const
           for (int u = 0; u < 8; ++u) {
             float4* a = reinterpret_cast<float4*>(rowp + ((static_cast<uint32_t>(u) ^ rsw) << 4));
             const float* x = acc + j * 32 + 4 * u;
-            const float4 o = *a;
-            *a = make_float4(fmaf(p.beta, o.x, p.alpha * x[0]), fmaf(p.beta, o.y, p.alpha * x[1]),
-                             fmaf(p.beta, o.z, p.alpha * x[2]), fmaf(p.beta, o.w, p.alpha * x[3]));
+            *a = make_float4(p.alpha * x[0], p.alpha * x[1], p.alpha * x[2], p.alpha * x[3]);
           }
         }
         // every epilogue thread takes the same branch (a lost wait stops all of them)
@@ -1032,7 +1018,7 @@ gptq_status launch_gemm_tc(const TcGemmArgs& g, cudaStream_t stream) {
                              tgp::BM, CU_TENSOR_MAP_SWIZZLE_128B)) != GPTQ_OK)
       return st;
     const int grid = p.n_tiles < num_sms() ? p.n_tiles : num_sms();
-    if (p.stage_c && !g.a_mn && g.b_mn && !g.lower && g.Cbig == nullptr && g.beta != 0.f &&
+    if (p.stage_c && !g.a_mn && g.b_mn && !g.lower && g.Cbig == nullptr && g.beta == 1.f &&
         g.N % tga::BN == 0) {
       // the lazy trailing update's shape: the A band stays in shared memory
       if ((st = set_max_dynamic_smem(reinterpret_cast<const void*>(gemm_tf32x3_aband_tc),
