@@ -40,7 +40,7 @@ typedef enum gptq_status {
   GPTQ_EINVAL = 1,         /* an argument is out of range, misaligned or inconsistent */
   GPTQ_ENOTPD = 2,         /* (from gptq_info_status) a factorization met a non-positive pivot */
   GPTQ_ECUDA = 3,          /* a CUDA runtime call failed (launch, attribute, driver entry point) */
-  GPTQ_EUNSUPPORTED = 4,   /* a valid request this build does not implement (e.g. dtype/size) */
+  GPTQ_EUNSUPPORTED = 4,   /* a valid request the library does not implement (e.g. dtype/size) */
   GPTQ_ETIMEOUT = 5,       /* (from gptq_info_status) a bounded device-side wait expired */
   GPTQ_EWORKSPACE = 6      /* workspace missing or smaller than gptq_workspace_size() */
 } gptq_status;
