@@ -258,6 +258,30 @@ __device__ __forceinline__ void diag_load_block(float* L, const float* A, int64_
   }
 }
 
+// Store rows [i0, i1) of the block: L when asked, and the tf32 split of the inverse (only its row
+// block and the ones left of it are nonzero). A warp per row (warps w0 .. w0 + nw - 1), the lanes
+// along it, so the shared-memory reads are conflict-free and every store covers 128 bytes.
+__device__ __forceinline__ void diag_store_rows(const float* L, const float* X, int i0, int i1,
+                                                int w0, int nw, float* A, int64_t lda, int k0,
+                                                int nb, float* Db, float* Ds, int64_t ldd,
+                                                int store_l) {
+  constexpr int NB = 128, LD = la::kLd;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = i0 + (warp - w0); i < i1 && i < nb; i += nw) {
+#pragma unroll
+    for (int u = 0; u < NB / 32; ++u) {
+      const int c = 32 * u + lane;
+      if (c < nb) {
+        const float x = (u <= (i >> 5)) ? X[i * LD + c] : 0.f;
+        const float bx = tf32_rna(x);
+        if (store_l) A[(k0 + i) * lda + k0 + c] = (c <= i) ? L[i * LD + c] : 0.f;
+        Db[i * ldd + c] = bx;
+        Ds[i * ldd + c] = x - bx;
+      }
+    }
+  }
+}
+
 // Factor and invert the block held in L (as diag_load_block leaves it): the tf32 split of its
 // inverse goes to (Db, Ds) with ld ldd, L itself to A[k0.., k0..] when store_l. stepA / stepX
 // (256 float4 each) and `bad` are shared scratch; the first pivot that was not positive is
@@ -316,6 +340,9 @@ __device__ __forceinline__ void diag_factor_block(float* sm, float4* stepA, floa
         named_barrier_or(la::kInverseBar, la::kInverseThreads, false);
       }
       if (kb >= 1) inverse_row_sum(L, X, OT + (kb & 1) * 32 * LDT, kb, first);
+      // row blocks 0-2 of the inverse (and rows 0-95 of L) are final now: store them while the
+      // last piece is factored
+      if (kb == 3) diag_store_rows(L, X, 0, 96, 4, 12, A, lda, k0, nb, Db, Ds, ldd, store_l);
     }
     __syncthreads();
     const int nbelow = NB - c0 - 32;
@@ -366,21 +393,8 @@ __device__ __forceinline__ void diag_factor_block(float* sm, float4* stepA, floa
   // the last row block of the inverse (its sums were formed alongside the last piece)
   inverse_row_product(X, OT + 1 * 32 * LDT, 3, 0);
   __syncthreads();
-  // store: L when asked, and the tf32 split of the inverse; a warp per row and the lanes along
-  // it, so the shared-memory reads are conflict-free and every store covers 128 bytes
-  for (int i = warp; i < nb; i += la::kDiagThreads / 32) {
-#pragma unroll
-    for (int u = 0; u < NB / 32; ++u) {
-      const int c = 32 * u + lane;
-      if (c < nb) {
-        const float x = (u <= (i >> 5)) ? X[i * LD + c] : 0.f;
-        const float bx = tf32_rna(x);
-        if (store_l) A[(k0 + i) * lda + k0 + c] = (c <= i) ? L[i * LD + c] : 0.f;
-        Db[i * ldd + c] = bx;
-        Ds[i * ldd + c] = x - bx;
-      }
-    }
-  }
+  // the last row block (rows 96 ..; the others were stored alongside the last piece)
+  diag_store_rows(L, X, 96, NB, 0, la::kDiagThreads / 32, A, lda, k0, nb, Db, Ds, ldd, store_l);
 }
 
 }  // namespace gptq
