@@ -27,8 +27,15 @@
 // in every CTA's list, so every wait ends while all CTAs of the grid (at most one per SM) are
 // resident; each wait is bounded in time all the same and reports GPTQ_INFO_TIMEOUT.
 //
-// Warps: 0 loads A/B by TMA, 1 issues the MMAs, 2 moves C boxes by TMA, 4-7 fold TMEM and write;
-// all 16 run the diagonal block's factorization on CTA 0 afterwards.
+// CTA 0 computes P(k+1) for itself only: its epilogue writes the split straight from TMEM into the
+// idle stage buffers, in the layout the MMA reads, and U(k+1, k+1) = A - L L^T multiplies that
+// split by itself without a trip through global memory; the update lands in the diagonal block's
+// shared layout (two warpgroups) and the factorization starts. CTA 1 computes the same P(k+1) as
+// its first panel tile, for global memory and the flag, so CTA 0 never waits for a store.
+//
+// Warps: 0 loads A/B by TMA, 1 issues the MMAs, 2 moves C boxes by TMA, 4-7 fold TMEM and write
+// (on CTA 0 also 8-11, for half of the diagonal block's update); all 16 run the diagonal block's
+// factorization on CTA 0 afterwards.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
