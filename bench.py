@@ -483,8 +483,10 @@ def bench_rotation(dev, stream, peaks, peaks_src, spec, X, iters=10):
     W = synth.weights_torch(spec, 1, dev).float()
     cases = [("calibration X %dx%d bf16 -> bf16" % tuple(X.shape), X, torch.empty_like(X)),
              ("weights W %dx%d fp32 -> fp32" % tuple(W.shape), W, torch.empty_like(W))]
-    out = {"kernel": "hadamard_rotate_kernel", "bound": "hbm", "peak_gbs": hbm,
-           "block": _lib.hadamard_block(spec.cols),
+    block = _lib.hadamard_block(spec.cols)
+    out = {"kernel": "hadamard4096_kernel" if block == 4096 else "hadamard_rotate_kernel",
+           "bound": "hbm", "peak_gbs": hbm,
+           "block": block,
            "peak_source": f"{peaks_src} HBM copy (kernel timed alone)", "cases": []}
     for name, src, dst in cases:
         for _ in range(3):

@@ -85,6 +85,32 @@ def test_rotate_in_place(n, rows):
     _check(X, Xd, signs)
 
 
+@pytest.mark.parametrize("xd,yd", [(torch.bfloat16, torch.bfloat16), (torch.float32, torch.float32)])
+def test_rotate_persistent_loop_every_row(xd, yd):
+    """2500 rows of order-4096 blocks: more segments than the persistent grid holds, so CTAs loop
+    (prefetching the next segment) with a ragged last round; every row against the oracle."""
+    rows, n = 2500, 4096
+    X = _input(rows, n, 14, xd)
+    signs = _signs(n, 15)
+    Y = torch.empty(rows, n, dtype=yd, device=DEV)
+    _lib.hadamard_rotate(X.to(DEV), Y, _sign_bits(signs))
+    torch.cuda.synchronize()
+    _check(X, Y, signs)
+
+
+@pytest.mark.parametrize("n", [49152, 69632])
+def test_rotate_many_blocks_per_row(n):
+    """12 blocks of 4096 per row (the fc2 input width; signs of the whole row in shared memory)
+    and 17 blocks (wider than the shared sign table: the three-pass kernel)."""
+    rows = 3
+    X = _input(rows, n, 16, torch.bfloat16)
+    signs = _signs(n, 17)
+    Y = torch.empty(rows, n, dtype=torch.bfloat16, device=DEV)
+    _lib.hadamard_rotate(X.to(DEV), Y, _sign_bits(signs))
+    torch.cuda.synchronize()
+    _check(X, Y, signs)
+
+
 def test_rotation_preserves_layer_products():
     """(W Q)(X Q)^T on the GPU outputs equals W X^T within the rounding of the two rotations."""
     rows, n, tokens = 16, 4096, 64
