@@ -112,6 +112,22 @@ __device__ __forceinline__ bool quantize_sub_block(float (&w4)[4], const float (
   return near;
 }
 
+// (a, a) as one 64-bit operand of the packed f32x2 instructions
+__device__ __forceinline__ uint64_t pair_of(float a) {
+  uint64_t p;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(p) : "f"(a));
+  return p;
+}
+
+// (x0, x1) <- (a0 * b0 + x0, a1 * b1 + x1), one packed f32x2 fused multiply-add (each lane rounds
+// once, as fmaf does)
+__device__ __forceinline__ void fma_x2(float& x0, float& x1, uint64_t a2, float b0, float b1) {
+  asm("{\n\t.reg .b64 b, c;\n\tmov.b64 b, {%3, %4};\n\tmov.b64 c, {%0, %1};\n\t"
+      "fma.rn.f32x2 c, %2, b, c;\n\tmov.b64 {%0, %1}, c;\n\t}"
+      : "+f"(x0), "+f"(x1)
+      : "l"(a2), "f"(b0), "f"(b1));
+}
+
 template <typename T>
 __device__ __forceinline__ float load_w(const T* p);
 template <>
@@ -381,7 +397,11 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
         qf[4 * t + u] = own ? rc4[u] + zq[u] : qf[4 * t + u];
         err[4 * t + u] = own ? e4[u] : err[4 * t + u];
       }
-      // the sub-block's errors on this lane's later columns (rank 4, one column after another)
+      // the sub-block's errors on this lane's later columns (rank 4, one column after another),
+      // two columns per packed multiply-add
+      uint64_t ne2[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) ne2[u] = pair_of(-e4[u]);
 #pragma unroll
       for (int t2 = t; t2 < NT; ++t2) {
         if (t2 == t && sub <= o) continue;   // earlier columns, or the sub-block itself
@@ -391,10 +411,8 @@ column_loop_kernel(float* __restrict__ Wh, int64_t rows, int64_t cols, const flo
           r[u] = *reinterpret_cast<const float4*>(Rz + (j0 + u) * B + S * t2 + 4 * sub);
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          v[4 * t2 + 0] = fmaf(-e4[u], r[u].x, v[4 * t2 + 0]);
-          v[4 * t2 + 1] = fmaf(-e4[u], r[u].y, v[4 * t2 + 1]);
-          v[4 * t2 + 2] = fmaf(-e4[u], r[u].z, v[4 * t2 + 2]);
-          v[4 * t2 + 3] = fmaf(-e4[u], r[u].w, v[4 * t2 + 3]);
+          fma_x2(v[4 * t2 + 0], v[4 * t2 + 1], ne2[u], r[u].x, r[u].y);
+          fma_x2(v[4 * t2 + 2], v[4 * t2 + 3], ne2[u], r[u].z, r[u].w);
         }
       }
     }
