@@ -31,6 +31,15 @@ namespace {
 // Packing
 // ------------------------------------------------------------------------------------------------
 
+// Eight codes (bytes of x: codes 0 .. 3, of y: codes 4 .. 7) -> one word whose byte i holds codes
+// 2i (low nibble) and 2i + 1 (high nibble).
+__device__ __forceinline__ uint32_t pack8_4bit(uint32_t x, uint32_t y) {
+  const uint32_t a = x & 0x0F0F0F0Fu, b = y & 0x0F0F0F0Fu;
+  const uint32_t even = __byte_perm(a, b, 0x6420);  // codes 0, 2, 4, 6
+  const uint32_t odd = __byte_perm(a, b, 0x7531);   // codes 1, 3, 5, 7
+  return even | (odd << 4);
+}
+
 // One thread per output word: eight consecutive codes of a row (8 bytes) -> one 32-bit word.
 __global__ void __launch_bounds__(256)
 pack_codes_4bit_kernel(const uint8_t* __restrict__ codes, int64_t rows, int64_t words_per_row,
@@ -43,12 +52,31 @@ pack_codes_4bit_kernel(const uint8_t* __restrict__ codes, int64_t rows, int64_t 
     const int64_t r = k / words_per_row, w = k - r * words_per_row;
     const uint2 v = __ldg(reinterpret_cast<const uint2*>(codes + r * ldc + 8 * w));
     bad |= ((v.x | v.y) & 0xF0F0F0F0u) != 0u;
-    // Bytes of v.x are codes 8w .. 8w+3, of v.y codes 8w+4 .. 8w+7. Word byte i must hold codes
-    // 2i (low nibble) and 2i+1 (high nibble).
-    const uint32_t a = v.x & 0x0F0F0F0Fu, b = v.y & 0x0F0F0F0Fu;
-    const uint32_t even = __byte_perm(a, b, 0x6420);  // codes 0, 2, 4, 6
-    const uint32_t odd = __byte_perm(a, b, 0x7531);   // codes 1, 3, 5, 7
-    packed[k] = even | (odd << 4);
+    packed[k] = pack8_4bit(v.x, v.y);
+  }
+  if (bad) record_info(info, GPTQ_INFO_BAD_CODE);
+  griddep_launch_dependents();
+}
+
+// One thread per 32 consecutive codes of a row (two 16-byte loads) -> four words (one 16-byte
+// store): cols % 32 == 0, ldc % 16 == 0 and both buffers 16-byte aligned.
+__global__ void __launch_bounds__(256)
+pack_codes_4bit_vec_kernel(const uint8_t* __restrict__ codes, int64_t rows,
+                           int64_t groups_per_row, int64_t ldc, uint32_t* __restrict__ packed,
+                           int32_t* info) {
+  griddep_wait();
+  const int64_t total = rows * groups_per_row;
+  bool bad = false;
+  for (int64_t k = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; k < total;
+       k += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = k / groups_per_row, gk = k - r * groups_per_row;
+    const uint4* src = reinterpret_cast<const uint4*>(codes + r * ldc + 32 * gk);
+    const uint4 p = __ldg(src), q = __ldg(src + 1);
+    bad |= ((p.x | p.y | p.z | p.w | q.x | q.y | q.z | q.w) & 0xF0F0F0F0u) != 0u;
+    // rows of the packed codes are dense: group gk of row r is 16-byte word k
+    reinterpret_cast<uint4*>(packed)[k] =
+        make_uint4(pack8_4bit(p.x, p.y), pack8_4bit(p.z, p.w), pack8_4bit(q.x, q.y),
+                   pack8_4bit(q.z, q.w));
   }
   if (bad) record_info(info, GPTQ_INFO_BAD_CODE);
   griddep_launch_dependents();
@@ -433,6 +461,13 @@ gptq_status launch_gemv(const CUtensorMap& tcodes, const CUtensorMap& tx, int xh
 
 gptq_status run_pack_codes_4bit(const uint8_t* codes, int64_t rows, int64_t cols, int64_t ldc,
                                 uint32_t* packed, int32_t* info, cudaStream_t stream) {
+  if (cols % 32 == 0 && ldc % 16 == 0 && (reinterpret_cast<uintptr_t>(codes) & 15u) == 0 &&
+      (reinterpret_cast<uintptr_t>(packed) & 15u) == 0) {
+    const int64_t total = rows * (cols / 32);
+    const int64_t blocks = std::min<int64_t>((total + 255) / 256, 16 * num_sms());
+    return launch_pdl(pack_codes_4bit_vec_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256),
+                      0, stream, codes, rows, cols / 32, ldc, packed, info);
+  }
   const int64_t words = rows * (cols / 8);
   int64_t blocks = (words + 255) / 256;
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;

@@ -81,8 +81,9 @@ def _check_matmul(codes, scales, zeros, group, X, rows_sel=None, ldx=None, ldy=N
 # packing
 # ---------------------------------------------------------------------------------------------
 
-@pytest.mark.parametrize("rows,cols", [(1, 8), (3, 64), (37, 4096), (129, 11008)])
+@pytest.mark.parametrize("rows,cols", [(1, 8), (5, 40), (3, 64), (37, 4096), (129, 11008)])
 def test_pack_bit_exact(rows, cols):
+    """Widths that are multiples of 32 take the 16-byte kernel, the others (8, 40) the word one."""
     codes, _, _ = synth.w4a16_operands_torch(rows, cols, -1, 11)
     packed, info = _pack_gpu(codes.to(DEV))
     assert info == 0
@@ -103,6 +104,20 @@ def test_pack_strided_input_and_bad_code():
     expect = codes.numpy().copy()
     expect[5, 17] = 0xA
     assert np.array_equal(_words_np(packed), oracle.pack_codes(expect))
+
+
+def test_pack_row_pitch_not_a_multiple_of_16():
+    """A row pitch of 264 bytes (8-byte aligned only) takes the word-at-a-time kernel."""
+    codes, _, _ = synth.w4a16_operands_torch(9, 256, -1, 13)
+    big = torch.zeros(9, 264, dtype=torch.uint8)
+    big[:, :256] = codes
+    dev = big.to(DEV)
+    packed = torch.empty(9, 32, dtype=torch.int32, device=DEV)
+    info = _info()
+    _lib.pack_codes_4bit(dev[:, :256], packed, info)
+    torch.cuda.synchronize()
+    assert int(info.item()) == 0
+    assert np.array_equal(_words_np(packed), oracle.pack_codes(codes.numpy()))
 
 
 def test_pack_of_gptq_codes():
