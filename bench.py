@@ -443,7 +443,7 @@ def bench_w4a16(dev, stream, peaks, peaks_src, iters=50):
 
     us = timed(fp, 20)
     nbytes = 1.5 * codes.numel()
-    out["pack"] = {"kernel": "pack_codes_4bit_kernel", "layer": "12288x49152", "us": us,
+    out["pack"] = {"kernel": "pack_codes_4bit_vec_kernel", "layer": "12288x49152", "us": us,
                    "bytes": nbytes, "achieved_gbs": nbytes / (us * 1e-6) / 1e9,
                    "frac": nbytes / (us * 1e-6) / 1e9 / hbm}
     # the 3-bit layout of the same layer's codes (values < 8): reads one byte per code, writes 3/8
