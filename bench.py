@@ -515,9 +515,11 @@ def bench_obq(dev, stream, rows=4096, cols=128, tokens=32768, iters=3):
     token-major bf16 inputs, H^-1 = R^T R in fp64. Times the OBQ kernel (greedy, and the natural
     order through the same downdates), and reports the proxy loss sum_r (w_hat - w)^T H_d
     (w_hat - w) of OBQ, of OBQ in natural order and of the library's GPTQ column loop, plus the
-    relative layer error with the undamped H. fp64 work per row ~ 2 cols^3 (the downdates);
-    the peak is derived, not measured: 148 SMs x 64 fp64 lanes x 1965 MHz = 18.6e12 fp64
-    instructions/s (the downdate's multiply and subtract are separate instructions)."""
+    relative layer error with the undamped H. fp64 work per row ~ 2 cols^3 instructions (the
+    downdates; their multiply and subtract are separate instructions). The peak is measured in
+    the same run: a cuBLAS fp64 GEMM's flop rate halved (one fused multiply-add per two flop) is
+    the fp64 instruction rate the GPU sustains; the nominal 148 SMs x 64 fp64 lanes x 1965 MHz =
+    18.6e12 instructions/s is kept beside it for context."""
     import torch
     from post_weight_quantization_12_b200 import _lib, synth
 
@@ -572,12 +574,17 @@ def bench_obq(dev, stream, rows=4096, cols=128, tokens=32768, iters=3):
         return float(((dW @ H) * dW).sum() / ((Wd @ H) * Wd).sum())
 
     fp64_ops = 2.0 * rows * cols ** 3
+    dgemm_tflops = measure_fp64_peak(dev)
+    peak = dgemm_tflops * 1e12 / 2.0
     out = {"layer": f"{rows}x{cols}, 4-bit per row, {tokens} bf16 tokens", "kernel": "obq_rows_kernel",
-           "bound": "alu", "peak": 18.6e12, "peak_unit": "fp64 instructions/s (derived, nominal)"}
+           "bound": "alu", "peak": peak,
+           "peak_unit": "fp64 instructions/s (measured: cuBLAS fp64 GEMM 4096^3, best of 5, "
+                        "flop rate / 2)",
+           "dgemm_tflops": dgemm_tflops, "nominal_peak": 18.6e12}
     for name, (ms, Wh) in outs.items():
         out[name] = {"ms": ms, "weights_per_s": rows * cols / (ms / 1e3),
                      "fp64_ops_per_s": fp64_ops / (ms / 1e3),
-                     "frac": fp64_ops / (ms / 1e3) / 18.6e12,
+                     "frac": fp64_ops / (ms / 1e3) / peak,
                      "proxy_loss": proxy(Wh), "rel_layer_error": rel_err(Wh)}
     out["gptq_column_loop"] = {"proxy_loss": proxy(W_g), "rel_layer_error": rel_err(W_g)}
     out["gptq_over_obq_proxy_loss"] = out["gptq_column_loop"]["proxy_loss"] / \
@@ -585,6 +592,30 @@ def bench_obq(dev, stream, rows=4096, cols=128, tokens=32768, iters=3):
     del X, S
     torch.cuda.empty_cache()
     return out
+
+
+def measure_fp64_peak(dev, n=4096, reps=5):
+    """Dense fp64 throughput on this GPU: torch.matmul of fp64 matrices (cuBLAS), n^3, best of
+    `reps` with CUDA events; 2 n^3 flop per product. Returns TFLOP/s."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(6)
+    a = torch.randn(n, n, device=dev, generator=g, dtype=torch.float64)
+    b = torch.randn(n, n, device=dev, generator=g, dtype=torch.float64)
+    c = torch.empty(n, n, device=dev, dtype=torch.float64)
+    for _ in range(2):
+        torch.matmul(a, b, out=c)
+    best = float("inf")
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch.matmul(a, b, out=c)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        best = min(best, e0.elapsed_time(e1))
+    del a, b, c
+    torch.cuda.empty_cache()
+    return 2.0 * n ** 3 / (best / 1e3) / 1e12
 
 
 def measure_tf32_peak(dev, n=8192, reps=10):
